@@ -1,0 +1,227 @@
+"""Plain CPU oracle of the H-BitLinear forward pass (BitNet v2).
+
+TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the benchmark's
+CPU-baseline leg may import this module. The product path (the CUDA library
+and its Python binding) never calls it and shares no code with it.
+
+It is written to be checked by eye against the sources, not to be fast:
+floating point in float64, integer matmul in int64, numpy library calls as
+single steps, no blocking or fusion beyond what the method states.
+
+Sources (the pages on the method; every formula on them was lost when the
+pages were extracted, the surrounding words survive):
+  [ABS]  "BitNet v2: Native 4-bit Activations with Hadamard Transformation
+         for 1-bit LLMs" (arXiv 2504.18415), abstract as shown on the
+         fugumt.com summary page.
+  [ART]  Chinese walkthrough of the BitNet v2 paper (m.jxzklqfsx.com,
+         article 817179), sections "BitNet v2：原生4位激活" and
+         "H-BitLinear模塊".
+  [B158] bitnet.cpp / BitNet b1.58 news article (gubiw.cn, 336601), section
+         "6 页论文，引入 1 bit LLM".
+
+Readings taken where the pages are silent or the formulas were dropped
+(each one is listed again with its reason in the design notes):
+  R1 weights: per-tensor absmean alpha = mean|W|; t = RoundClip(W/(alpha+eps_w), -1, 1).
+  R2 norm: RMSNorm over the K features of a token, x / sqrt(mean(x^2) + eps_n),
+     optional per-feature gain; eps_n defaults to 1e-6.
+  R3 transform: Sylvester-ordered Walsh-Hadamard matrix scaled by 1/sqrt(n)
+     (orthonormal); when K is not a power of two, the same transform is applied
+     to each consecutive block of n features (block-diagonal).
+  R4 activation quantisers, per token row:
+       a8 absmax : gamma = max|x|, q = RoundClip(127 x/(gamma+eps), -128, 127), s = gamma/127
+       a4 absmean: beta = mean|x|, q = RoundClip(sqrt7 x/(beta+eps), -8, 7), s = beta/sqrt7
+       a4 absmax : gamma = max|x|, q = RoundClip(7 x/(gamma+eps), -8, 7),    s = gamma/7
+     A row whose statistic is zero (and eps = 0) gives q = 0 and s = 0.
+  R5 RoundClip rounds to nearest, ties to even. The rounding decision is taken
+     on float32 operands in float32 (the precision the GPU kernel decides in):
+     the element and the per-row multiplier are rounded to float32, multiplied
+     in float32, then rounded to an integer. Everything before that is float64.
+  R6 output: y[m, n] = s[m] * alpha * sum_k q[m, k] t[k, n], evaluated in float64.
+
+Parity status: the transform, the quantisers, the ternariser and the integer
+product are pinned by the tests (closed forms, a dense Sylvester matrix from
+SciPy, brute force on small inputs, a hand-derived worked example). The
+choice of readings R1-R6 themselves is not pinned by any number on the pages,
+which print none: against the published method the oracle is "parity
+unpinned" in that sense only.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+SQRT7 = math.sqrt(7.0)
+
+__all__ = [
+    "bf16_to_f64",
+    "absmean_ternarize",
+    "rmsnorm",
+    "fwht",
+    "hadamard_transform",
+    "quantize",
+    "norm_fht_quant",
+    "ternary_matmul",
+    "dequant",
+    "h_bitlinear_forward",
+]
+
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> float64, exactly (bf16 is the top half of a float32)."""
+    b = np.asarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def absmean_ternarize(W: np.ndarray, eps_w: float = 0.0) -> tuple[np.ndarray, float]:
+    """Per-tensor absmean ternarisation of the weights (reading R1).
+
+    [ART] "H-BitLinear模塊": the weights are ternarised to {-1, 0, 1} with a
+    per-tensor absmean scale. [B158] "6 页论文，引入 1 bit LLM": the weight
+    matrix is scaled by its mean absolute value and each entry is rounded to the
+    nearest of -1, 0, 1.
+
+    Returns (t int8 with the shape of W, alpha). The rounding decision uses
+    float64 (the weight packer on the GPU also decides in float64).
+    """
+    W = np.asarray(W, dtype=np.float64)
+    alpha = float(np.sum(np.abs(W)) / W.size)
+    denom = alpha + eps_w
+    if denom == 0.0:
+        return np.zeros(W.shape, dtype=np.int8), alpha
+    t = np.clip(np.rint(W / denom), -1, 1).astype(np.int8)
+    return t, alpha
+
+
+def rmsnorm(x: np.ndarray, gain: np.ndarray | None = None, eps: float = 1e-6) -> np.ndarray:
+    """RMSNorm of each row over its K features (reading R2).
+
+    [ART] "BitNet v2：原生4位激活": the model is built from LLaMA-like parts
+    including RMS normalisation; "H-BitLinear模塊" names the normalisation
+    applied inside the layer before the Hadamard transform.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    r = np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    y = x / r
+    if gain is not None:
+        y = y * np.asarray(gain, dtype=np.float64)
+    return y
+
+
+def fwht(x: np.ndarray) -> np.ndarray:
+    """Orthonormal fast Walsh-Hadamard transform along the last axis (reading R3).
+
+    [ART] "H-BitLinear模塊": the product with the Hadamard matrix is computed by
+    the fast Hadamard transform in O(n log n); the matrix has entries +-1 and
+    mutually orthogonal rows. This is the Sylvester construction
+    H_2n = [[H_n, H_n], [H_n, -H_n]], realised as log2(n) butterfly stages: at
+    stage h the pair (x[j], x[j+h]) inside each block of 2h becomes
+    (x[j] + x[j+h], x[j] - x[j+h]). The result is scaled by 1/sqrt(n).
+    """
+    y = np.array(x, dtype=np.float64, copy=True)
+    n = y.shape[-1]
+    if n < 1 or n & (n - 1):
+        raise ValueError(f"transform length {n} is not a power of two")
+    lead = y.shape[:-1]
+    h = 1
+    while h < n:
+        v = y.reshape(*lead, n // (2 * h), 2, h)
+        a = v[..., 0, :].copy()
+        b = v[..., 1, :].copy()
+        v[..., 0, :] = a + b
+        v[..., 1, :] = a - b
+        h *= 2
+    return y / math.sqrt(n)
+
+
+def hadamard_transform(x: np.ndarray, block: int = 0) -> np.ndarray:
+    """Hadamard transform of each row: over all of K (block = 0) or block-diagonal.
+
+    Block-diagonal (reading R3): K = nb * block, and each consecutive slice of
+    `block` features is transformed on its own, i.e. the matrix is
+    kron(I_nb, H_block / sqrt(block)).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    K = x.shape[-1]
+    if block == 0 or block == K:
+        return fwht(x)
+    if K % block:
+        raise ValueError(f"K={K} is not a multiple of block={block}")
+    lead = x.shape[:-1]
+    return fwht(x.reshape(*lead, K // block, block)).reshape(*lead, K)
+
+
+def _round_clip_f32(x: np.ndarray, mult: np.ndarray, lo: int, hi: int) -> np.ndarray:
+    """RoundClip with the decision taken in float32 (reading R5)."""
+    v = x.astype(np.float32) * mult.astype(np.float32)  # float32 product of float32 operands
+    return np.clip(np.rint(v), lo, hi).astype(np.int8)  # ties to even
+
+
+def quantize(xr: np.ndarray, abits: int, scale_mode: str, eps_q: float = 0.0
+             ) -> tuple[np.ndarray, np.ndarray]:
+    """Per-token activation quantisation without zero point (reading R4).
+
+    [ART] "H-BitLinear模塊": separate strategies for INT8 and INT4 activations
+    (formulas dropped in extraction). [B158] "6 页论文，引入 1 bit LLM":
+    activations are scaled into [-Q_b, Q_b], which removes the zero point.
+
+    Returns (q int8 [M, K], s float64 [M]).
+    """
+    xr = np.asarray(xr, dtype=np.float64)
+    a = np.abs(xr)
+    if abits == 8 and scale_mode == "absmax":
+        stat, qmul, lo, hi = a.max(axis=-1), 127.0, -128, 127
+    elif abits == 4 and scale_mode == "absmean":
+        stat, qmul, lo, hi = a.mean(axis=-1), SQRT7, -8, 7
+    elif abits == 4 and scale_mode == "absmax":
+        stat, qmul, lo, hi = a.max(axis=-1), 7.0, -8, 7
+    else:
+        raise ValueError(f"unsupported quantiser abits={abits} scale_mode={scale_mode!r}")
+    denom = stat + eps_q
+    live = denom > 0.0
+    mult = np.where(live, qmul / np.where(live, denom, 1.0), 0.0)
+    q = _round_clip_f32(xr, mult[..., None], lo, hi)
+    s = np.where(live, stat / qmul, 0.0)
+    return q, s
+
+
+def norm_fht_quant(x: np.ndarray, gain: np.ndarray | None, had_block: int, abits: int,
+                   scale_mode: str, eps_norm: float = 1e-6, eps_q: float = 0.0
+                   ) -> tuple[np.ndarray, np.ndarray]:
+    """Activation side of H-BitLinear: Q(Hadamard(RMSNorm(x))) per token row.
+
+    [ABS]: an online Hadamard transformation is applied before activation
+    quantisation. [ART] "H-BitLinear模塊": the layer computes
+    Q_w(W) . Q_INT8/INT4(Hadamard(LN(X))).
+
+    x: float64 values (or bf16 bit patterns as uint16) [M, K].
+    """
+    if x.dtype == np.uint16:
+        x = bf16_to_f64(x)
+    xr = hadamard_transform(rmsnorm(x, gain, eps_norm), had_block)
+    return quantize(xr, abits, scale_mode, eps_q)
+
+
+def ternary_matmul(q: np.ndarray, t: np.ndarray) -> np.ndarray:
+    """acc[m, n] = sum_k q[m, k] * t[k, n] in exact int64 arithmetic."""
+    return np.asarray(q, dtype=np.int64) @ np.asarray(t, dtype=np.int64)
+
+
+def dequant(acc: np.ndarray, s: np.ndarray, alpha: float) -> np.ndarray:
+    """y[m, n] = acc[m, n] * s[m] * alpha in float64 (reading R6)."""
+    return np.asarray(acc, dtype=np.float64) * np.asarray(s, dtype=np.float64)[:, None] * float(alpha)
+
+
+def h_bitlinear_forward(x: np.ndarray, W: np.ndarray, gain: np.ndarray | None = None,
+                        had_block: int = 0, abits: int = 4, scale_mode: str | None = None,
+                        eps_norm: float = 1e-6, eps_q: float = 0.0, eps_w: float = 0.0) -> dict:
+    """The whole layer: weights ternarised, activations normed/rotated/quantised, product, dequant.
+
+    Returns a dict with every intermediate (t, alpha, q, s, acc, y) for parity checks.
+    """
+    if scale_mode is None:
+        scale_mode = "absmax" if abits == 8 else "absmean"
+    t, alpha = absmean_ternarize(W, eps_w)
+    q, s = norm_fht_quant(x, gain, had_block, abits, scale_mode, eps_norm, eps_q)
+    acc = ternary_matmul(q, t)
+    return {"t": t, "alpha": alpha, "q": q, "s": s, "acc": acc, "y": dequant(acc, s, alpha)}

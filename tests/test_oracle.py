@@ -1,0 +1,287 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test checks one part of the oracle against a closed form, a library
+routine of different construction (SciPy's Sylvester Hadamard matrix, float64
+BLAS), brute force, or the hand-derived worked example in tests/golden. The
+mutation tests at the end plant plausible mistakes in the oracle and check
+that at least one pin catches each.
+"""
+import math
+
+import numpy as np
+import pytest
+import scipy.linalg
+
+import conftest
+import oracle
+from hadamard_bit_quant_hbl_b200 import inputs
+
+RNG = np.random.default_rng(12345)
+
+
+# ---------------------------------------------------------------- transform
+
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 64, 256, 1024])
+def test_fwht_equals_scipy_sylvester_matrix(n):
+    # fwht of the identity rows gives the columns of H_n / sqrt(n); SciPy builds H_n by the
+    # Sylvester recursion directly (no butterflies).
+    got = oracle.fwht(np.eye(n))
+    want = scipy.linalg.hadamard(n).astype(np.float64) / math.sqrt(n)
+    np.testing.assert_allclose(got, want.T, rtol=0, atol=1e-12)
+
+
+def test_fwht_walsh_closed_form():
+    # Sylvester-ordered Hadamard entry: H[i, j] = (-1)^popcount(i & j).
+    n = 4096
+    for j in RNG.integers(0, n, size=6):
+        e = np.zeros(n)
+        e[j] = 1.0
+        got = oracle.fwht(e) * math.sqrt(n)
+        i = np.arange(n)
+        want = np.array([(-1.0) ** bin(int(ii) & int(j)).count("1") for ii in i])
+        np.testing.assert_array_equal(got, want)
+
+
+def test_fwht_orthogonal_involution_parseval():
+    n = 8192
+    x = RNG.standard_normal((3, n))
+    y = oracle.fwht(x)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12)
+    np.testing.assert_allclose(oracle.fwht(y), x, rtol=0, atol=1e-11)
+    # H H^T = n I, exactly in integers, on a 256-point matrix built by the oracle
+    H = np.rint(oracle.fwht(np.eye(256)) * 16).astype(np.int64)
+    np.testing.assert_array_equal(H @ H.T, 256 * np.eye(256, dtype=np.int64))
+
+
+def test_fwht_delta_and_constant():
+    n = 2048
+    e0 = np.zeros(n)
+    e0[0] = 1
+    np.testing.assert_allclose(oracle.fwht(e0), np.full(n, 1 / math.sqrt(n)), rtol=1e-13)
+    np.testing.assert_allclose(oracle.fwht(np.ones(n)), math.sqrt(n) * e0, atol=1e-11)
+
+
+def test_fwht_rejects_non_power_of_two():
+    with pytest.raises(ValueError):
+        oracle.fwht(np.ones(12))
+
+
+def test_block_diagonal_transform_matches_kron():
+    blk = 256
+    nb = 6
+    x = RNG.standard_normal((4, nb * blk))
+    dense = np.kron(np.eye(nb), scipy.linalg.hadamard(blk) / 16.0)
+    np.testing.assert_allclose(oracle.hadamard_transform(x, blk), x @ dense.T, atol=1e-12)
+    # 43 blocks (K = 11008), checked block by block against the dense 256-point matrix
+    x = RNG.standard_normal((2, 43 * blk))
+    got = oracle.hadamard_transform(x, blk)
+    H = scipy.linalg.hadamard(blk) / 16.0
+    for b in range(43):
+        sl = slice(b * blk, (b + 1) * blk)
+        np.testing.assert_allclose(got[:, sl], x[:, sl] @ H.T, atol=1e-12)
+
+
+# ---------------------------------------------------------------- norm
+
+def test_rmsnorm_unit_rms_and_gain():
+    x = RNG.laplace(0, 0.1, size=(5, 512))
+    y = oracle.rmsnorm(x, None, eps=0.0)
+    np.testing.assert_allclose(np.sqrt(np.mean(y ** 2, axis=1)), 1.0, rtol=1e-13)
+    # the output is x divided by a positive per-row factor
+    ratio = y / x
+    np.testing.assert_allclose(ratio, ratio[:, :1] * np.ones_like(ratio), rtol=1e-12)
+    g = RNG.uniform(0.5, 2.0, size=512)
+    np.testing.assert_allclose(oracle.rmsnorm(x, g, eps=0.0), y * g, rtol=1e-13)
+    # eps enters under the square root: a zero row stays zero
+    np.testing.assert_array_equal(oracle.rmsnorm(np.zeros((1, 8)), None, 1e-6), np.zeros((1, 8)))
+
+
+def test_rms_is_preserved_by_the_orthonormal_transform():
+    x = RNG.standard_normal((3, 1024))
+    np.testing.assert_allclose(np.mean(oracle.fwht(x) ** 2, axis=1), np.mean(x ** 2, axis=1), rtol=1e-12)
+
+
+# ---------------------------------------------------------------- quantisers
+
+QUANTS = [(8, "absmax", 127, -128, 127), (4, "absmean", math.sqrt(7), -8, 7), (4, "absmax", 7, -8, 7)]
+
+
+@pytest.mark.parametrize("abits,mode,Q,lo,hi", QUANTS)
+def test_quantiser_defining_properties(abits, mode, Q, lo, hi):
+    x = RNG.laplace(0, 1.0, size=(64, 256))
+    x[:, 7] *= 30  # an outlier channel
+    q, s = oracle.quantize(x, abits, mode)
+    assert q.dtype == np.int8 and q.min() >= lo and q.max() <= hi
+    a = np.abs(x)
+    # the scale is the row statistic divided by the code range, computed independently here
+    stat = a.max(axis=1) if mode == "absmax" else a.sum(axis=1) / a.shape[1]
+    np.testing.assert_allclose(s * Q, stat, rtol=1e-13)
+    # rounding to nearest: every unclipped code is within half a step of x / s
+    v = x / s[:, None]
+    unclipped = (v > lo - 0.5) & (v < hi + 0.5)
+    assert np.all(np.abs(v[unclipped] - q[unclipped]) <= 0.5 + 1e-5)
+    # clipped codes sit at the bound on the correct side
+    assert np.all(q[v >= hi + 0.5] == hi) and np.all(q[v <= lo - 0.5] == lo)
+    if mode == "absmax":
+        # the largest magnitude maps to +-Q exactly
+        am = np.argmax(a, axis=1)
+        np.testing.assert_array_equal(np.abs(q[np.arange(64), am]), int(Q))
+
+
+@pytest.mark.parametrize("abits,mode,Q,lo,hi", QUANTS)
+def test_quantiser_brute_force_nearest_code(abits, mode, Q, lo, hi):
+    # brute force: among all codes in [lo, hi] the oracle picks the one nearest to the
+    # float32 value it decides on (ties to the even code).
+    x = RNG.standard_normal((8, 32))
+    q, s = oracle.quantize(x, abits, mode)
+    stat = np.abs(x).max(axis=1) if mode == "absmax" else np.abs(x).mean(axis=1)
+    for m in range(8):
+        mult = np.float32(Q / stat[m])
+        for k in range(32):
+            vv = float(np.float32(x[m, k]) * mult)
+            best = min(range(lo, hi + 1), key=lambda c: (abs(vv - c), c % 2))
+            assert q[m, k] == best, (m, k, vv, q[m, k], best)
+
+
+def test_quantiser_zero_row_and_scale_invariance():
+    x = np.zeros((2, 64))
+    x[1] = RNG.standard_normal(64)
+    for abits, mode, *_ in QUANTS:
+        q, s = oracle.quantize(x, abits, mode)
+        assert np.all(q[0] == 0) and s[0] == 0.0
+        q4, s4 = oracle.quantize(4.0 * x, abits, mode)  # power of two: exact scaling
+        np.testing.assert_array_equal(q4, q)
+        np.testing.assert_array_equal(s4, 4.0 * s)
+
+
+def test_quantiser_rejects_unknown_modes():
+    with pytest.raises(ValueError):
+        oracle.quantize(np.ones((1, 4)), 8, "absmean")
+    with pytest.raises(ValueError):
+        oracle.quantize(np.ones((1, 4)), 2, "absmax")
+
+
+# ---------------------------------------------------------------- weights
+
+def test_ternarize_constant_and_brute_force():
+    for c in (0.3, -0.07):
+        t, alpha = oracle.absmean_ternarize(np.full((4, 6), c))
+        assert alpha == pytest.approx(abs(c), rel=1e-15)
+        np.testing.assert_array_equal(t, np.sign(c) * np.ones((4, 6)))
+    W = RNG.standard_normal((16, 8)) * 0.02
+    t, alpha = oracle.absmean_ternarize(W)
+    assert set(np.unique(t)) <= {-1, 0, 1}
+    assert alpha == pytest.approx(np.abs(W).sum() / W.size, rel=1e-14)
+    for (k, n), w in np.ndenumerate(W):
+        best = min((-1, 0, 1), key=lambda c: abs(w / alpha - c))
+        assert t[k, n] == best
+    t0, a0 = oracle.absmean_ternarize(np.zeros((3, 3)))
+    assert a0 == 0.0 and not t0.any()
+
+
+# ---------------------------------------------------------------- product
+
+def test_ternary_matmul_brute_force_and_blas():
+    q = RNG.integers(-8, 8, size=(5, 37)).astype(np.int8)
+    t = RNG.integers(-1, 2, size=(37, 6)).astype(np.int8)
+    acc = oracle.ternary_matmul(q, t)
+    for m in range(5):
+        for n in range(6):
+            assert acc[m, n] == sum(int(q[m, k]) * int(t[k, n]) for k in range(37))
+    # float64 BLAS is exact here (integers far below 2^53), and computes in another order
+    q = RNG.integers(-128, 128, size=(64, 4096)).astype(np.int8)
+    t = RNG.integers(-1, 2, size=(4096, 48)).astype(np.int8)
+    np.testing.assert_array_equal(oracle.ternary_matmul(q, t),
+                                  (q.astype(np.float64) @ t.astype(np.float64)).astype(np.int64))
+
+
+# ---------------------------------------------------------------- worked example
+
+@pytest.mark.parametrize("abits,mode,key", [(8, "absmax", "a8"), (4, "absmean", "a4_absmean"),
+                                            (4, "absmax", "a4_absmax")])
+def test_worked_example(golden, abits, mode, key):
+    g = golden("worked_example_k4.txt")
+    x = np.array([g["x"]])
+    W = np.array(g["W"]).reshape(4, 2)
+    out = oracle.h_bitlinear_forward(x, W, None, 0, abits, mode, eps_norm=0.0)
+    xr = oracle.hadamard_transform(oracle.rmsnorm(x, None, 0.0))
+    np.testing.assert_allclose(xr[0], g["xr"], rtol=1e-14, atol=1e-15)
+    np.testing.assert_array_equal(out["t"].ravel(), np.array(g["t"]))
+    assert out["alpha"] == pytest.approx(g["alpha"][0], rel=1e-14)
+    np.testing.assert_array_equal(out["q"][0], np.array(g[f"{key}_q"]))
+    assert out["s"][0] == pytest.approx(g[f"{key}_s"][0], rel=1e-13)
+    np.testing.assert_array_equal(out["acc"][0], np.array(g[f"{key}_acc"]))
+    np.testing.assert_allclose(out["y"][0], g[f"{key}_y"], rtol=1e-13)
+
+
+# ---------------------------------------------------------------- whole layer
+
+def test_forward_equals_dense_dequantised_product():
+    # The layer's output written the way the method states it, Q_w(W) . Q(Hadamard(LN(X))),
+    # with dense matrices: dequantised activations times dequantised weights.
+    K, N, M = 512, 24, 9
+    x = RNG.laplace(0, 0.05, size=(M, K))
+    x[:, 3] *= 50
+    W = RNG.standard_normal((K, N)) * 0.02
+    out = oracle.h_bitlinear_forward(x, W, None, 0, 4, "absmean")
+    xn = x / np.sqrt((x ** 2).mean(axis=1, keepdims=True) + 1e-6)
+    xr = xn @ (scipy.linalg.hadamard(K) / math.sqrt(K)).T
+    np.testing.assert_allclose(xr, oracle.hadamard_transform(oracle.rmsnorm(x)), atol=1e-12)
+    Xq = out["q"].astype(np.float64) * out["s"][:, None]
+    Wq = out["t"].astype(np.float64) * out["alpha"]
+    np.testing.assert_allclose(out["y"], Xq @ Wq, rtol=1e-12, atol=1e-14)
+
+
+def test_transform_flattens_outliers_on_workload_inputs():
+    # Property of the method (BitNet v2 abstract; walkthrough Figs. 2-3): after the transform
+    # the outlier-heavy activations are far less heavy-tailed. Sanity only, not parity.
+    spec = inputs.WORKLOADS["wo_1p3b_a4"].with_m(32)
+    x = oracle.bf16_to_f64(inputs.activations(spec))
+
+    def kurt(a):
+        a = a - a.mean(axis=1, keepdims=True)
+        return np.mean(a ** 4, axis=1) / np.mean(a ** 2, axis=1) ** 2
+
+    xr = oracle.hadamard_transform(oracle.rmsnorm(x))
+    assert np.median(kurt(x)) > 20 * np.median(kurt(xr))
+    assert np.median(kurt(xr)) < 4.0
+
+
+# ---------------------------------------------------------------- planted mistakes
+
+_REAL_FWHT = oracle.fwht
+
+
+def _fwht_no_scale(x):
+    return _REAL_FWHT(x) * math.sqrt(np.asarray(x).shape[-1])
+
+
+def _fwht_reversed_order(x):
+    return _REAL_FWHT(x)[..., ::-1].copy()
+
+
+@pytest.mark.parametrize("mutant", [_fwht_no_scale, _fwht_reversed_order])
+def test_planted_transform_mistakes_are_caught(monkeypatch, mutant):
+    monkeypatch.setattr(oracle.hbl_oracle, "fwht", mutant)
+    monkeypatch.setattr(oracle, "fwht", mutant)
+    caught = 0
+    for check in (lambda: test_fwht_equals_scipy_sylvester_matrix(8),
+                  lambda: test_worked_example(conftest.load_golden, 8, "absmax", "a8")):
+        try:
+            check()
+        except AssertionError:
+            caught += 1
+    assert caught >= 1
+
+
+def test_planted_quantiser_mistake_is_caught(monkeypatch):
+    real = oracle.hbl_oracle.quantize
+
+    def floor_instead_of_round(xr, abits, mode, eps_q=0.0):
+        q, s = real(xr, abits, mode, eps_q)
+        v = np.asarray(xr) / np.where(s > 0, s, 1)[:, None]
+        return np.clip(np.floor(v), -8 if abits == 4 else -128, 7 if abits == 4 else 127).astype(np.int8), s
+
+    monkeypatch.setattr(oracle, "quantize", floor_instead_of_round)
+    with pytest.raises(AssertionError):
+        test_quantiser_defining_properties(4, "absmean", math.sqrt(7), -8, 7)
