@@ -1,0 +1,368 @@
+#!/usr/bin/env python3
+"""Benchmark of the H-BitLinear forward pass (BitNet v2) on B200.
+
+One step = the hot path over one batch: RMSNorm -> Hadamard -> a4 quantisation -> ternary
+product -> dequant, for both H-BitLinear layers of a 7B-like block (attention output Wo 4096->4096
+and FFN down Wdown 16384->4096) at 8192 tokens. Weights are packed once before timing (offline).
+Activations are synthetic (seeded Laplace body + 1% outlier channels x50, bf16).
+
+Prints one JSON line (rank 0). `--impl reference` times the CPU oracle instead, on a bounded
+sample of the same workload.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  (N > 1: launched by torch.distributed.run; every rank runs an independent replica)
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hadamard_bit_quant_hbl_b200 import inputs  # noqa: E402
+
+METRIC = "H-BitLinear tokens/s and effective TOPS at 7B-like shapes; % of HBM/int8 roofline"
+UNIT = "tokens/s"
+M_TOKENS = 8192
+LAYERS = ("wo_7b_a4", "wdown_7b_a4")
+WORKLOAD = ("7B-like H-BitLinear layer pair: Wo 4096->4096 + Wdown 16384->4096, a4 absmean, "
+            "8192 tokens, bf16 in / bf16 out")
+# DRAM bytes per launch of the dominant kernel from an ncu capture, with the hash of the kernel
+# source it was taken on (reported as null once the source has changed).
+NCU_TRAFFIC = {}
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], p["bf16_tflops_sustained"], "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def src_hash(name):
+    with open(os.path.join(ROOT, "hadamard_bit_quant_hbl_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML (read-only) while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            phys = int(vis.split(",")[device_index]) if vis and vis.split(",")[0].isdigit() else device_index
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(phys)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            pass
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+# ---------------------------------------------------------------- CPU oracle (reference arm)
+
+def oracle_prepare(rows_per_layer):
+    """Inputs of the oracle sample: the first `rows_per_layer` token rows of each layer, with the
+    weights ternarised beforehand (offline, like the GPU path)."""
+    import oracle
+
+    prepared = []
+    for name in LAYERS:
+        spec = inputs.WORKLOADS[name].with_m(rows_per_layer)
+        t, alpha = oracle.absmean_ternarize(inputs.weights(spec))
+        prepared.append((spec, inputs.activations(spec), t, alpha))
+    return prepared
+
+
+def oracle_step(prepared):
+    """One oracle pass of S1-S5 over the prepared rows of both layers; returns seconds."""
+    import oracle
+
+    t0 = time.perf_counter()
+    for spec, x, t, alpha in prepared:
+        q, s = oracle.norm_fht_quant(x, None, spec.had_block, 4, "absmean")
+        oracle.dequant(oracle.ternary_matmul(q, t), s, alpha)
+    return time.perf_counter() - t0
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    rows = max(1, args.ref_step_rows)
+    prepared = oracle_prepare(rows)
+    for _ in range(args.warmup):
+        oracle_step(prepared)
+    times = [oracle_step(prepared) for _ in range(args.steps)]
+    t = sum(times) / len(times)
+    value = rows / t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64/int64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": M_TOKENS, "sample_rows_per_layer": rows},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"first {rows} token rows of each layer per step, S1-S5 "
+                                   "(weights ternarised before timing)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    import hadamard_bit_quant_hbl_b200 as hbl
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    layers = []
+    for name in LAYERS:
+        spec = inputs.WORKLOADS[name].with_m(M_TOKENS)
+        x = inputs.activations(spec)
+        W = torch.from_numpy(inputs.weights(spec)).to(dev)
+        packed, alpha = hbl.hbl_pack_weights(W)
+        del W
+        X = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+        Xh = torch.from_numpy(x.view(np.int16)).pin_memory()
+        fmt = hbl.HBL_CODES_I8
+        codes = torch.empty((spec.M, spec.K), dtype=torch.uint8, device=dev)
+        s_x = torch.empty(spec.M, dtype=torch.float32, device=dev)
+        Y = torch.empty((spec.M, spec.N), dtype=torch.bfloat16, device=dev)
+        Yh = torch.empty((spec.M, spec.N), dtype=torch.bfloat16).pin_memory()
+        ws = torch.empty(hbl.hbl_forward_workspace(spec.M, spec.K, hbl.HBL_Q_A4_ABSMEAN), dtype=torch.uint8, device=dev)
+        layers.append(dict(spec=spec, X=X, Xh=Xh, packed=packed, alpha=alpha, codes=codes, s_x=s_x, Y=Y, Yh=Yh,
+                           ws=ws, fmt=fmt))
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+
+    def step(ev=None):
+        for i, L in enumerate(layers):
+            sp = L["spec"]
+            hbl.hbl_norm_fht_quant(L["X"], None, sp.had_block, hbl.HBL_Q_A4_ABSMEAN, 1e-6, 0.0, L["fmt"], L["codes"],
+                                   L["s_x"], stream=sh)
+            if ev is not None:
+                ev[2 * i].record(stream)
+            hbl.hbl_ternary_gemm(L["codes"], L["fmt"], 4, L["s_x"], L["packed"], L["alpha"], sp.N, sp.K, L["Y"],
+                                 hbl.HBL_OUT_BF16, None, stream=sh)
+            if ev is not None:
+                ev[2 * i + 1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = hbl.hbl_device_status()
+    if st != hbl.HBL_OK:
+        raise RuntimeError(hbl.hbl_status_string(st))
+
+    # ---- timed region: exactly K steps, events between every kernel pair
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for k in range(args.steps):
+            step(evs[k])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total_ms = start.elapsed_time(evs[-1][-1])
+    # per-kernel averages: [nfq Wo, gemm Wo, nfq Wdown, gemm Wdown]
+    per = np.zeros(4)
+    for k in range(args.steps):
+        prev = start if k == 0 else evs[k - 1][3]
+        marks = [prev] + evs[k]
+        for j in range(4):
+            per[j] += marks[j].elapsed_time(marks[j + 1])
+    per /= args.steps
+    # per-kernel split of the first pair includes the launch of the nfq kernel of layer 0 only
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_step = total_ms / args.steps
+    tokens = M_TOKENS * world
+    value = tokens / (ms_step / 1e3)
+
+    # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        for L in layers:
+            L["X"].copy_(L["Xh"].view(torch.bfloat16), non_blocking=True)
+            hbl.hbl_forward(L["X"], L["packed"], L["alpha"], L["spec"].N, None, L["spec"].had_block,
+                            hbl.HBL_Q_A4_ABSMEAN, workspace=L["ws"], Y=L["Y"], out_dtype=hbl.HBL_OUT_BF16, stream=sh)
+            L["Yh"].copy_(L["Y"], non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for L in layers:
+            L["X"].copy_(L["Xh"].view(torch.bfloat16), non_blocking=True)
+            hbl.hbl_forward(L["X"], L["packed"], L["alpha"], L["spec"].N, None, L["spec"].had_block,
+                            hbl.HBL_Q_A4_ABSMEAN, workspace=L["ws"], Y=L["Y"], out_dtype=hbl.HBL_OUT_BF16, stream=sh)
+            L["Yh"].copy_(L["Y"], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = sum(L["X"].numel() * 2 for L in layers)
+    d2h = sum(L["Y"].numel() * 2 for L in layers)
+
+    st = hbl.hbl_device_status()
+    if st != hbl.HBL_OK:
+        raise RuntimeError(hbl.hbl_status_string(st))
+    if rank != 0:
+        return
+
+    hbm, bf16, bf16_sus, peak_src = peaks()
+    int8_peak_tops = 2.0 * bf16_sus  # nominal dense int8 : bf16 ratio 4.5 : 2.25 PFLOP/s
+    kern = []
+    for i, L in enumerate(layers):
+        sp = L["spec"]
+        nfq_bytes = 2 * sp.M * sp.K + sp.M * sp.K + 4 * sp.M
+        gemm_ops = 2.0 * sp.M * sp.N * sp.K
+        kern.append({"kernel": f"norm_fht_quant[{sp.name}]", "ms": per[2 * i], "bound": "hbm",
+                     "achieved": nfq_bytes / (per[2 * i] / 1e3) / 1e9, "unit": "GB/s",
+                     "frac": nfq_bytes / (per[2 * i] / 1e3) / 1e9 / hbm})
+        kern.append({"kernel": f"gemm_tc[{sp.name}]", "ms": per[2 * i + 1], "bound": "tensor",
+                     "achieved": gemm_ops / (per[2 * i + 1] / 1e3) / 1e12, "unit": "TOP/s",
+                     "frac": gemm_ops / (per[2 * i + 1] / 1e3) / 1e12 / int8_peak_tops})
+    dom = max(kern, key=lambda k: k["ms"])
+    traffic = None
+    rec = NCU_TRAFFIC.get(dom["kernel"])
+    if rec and rec.get("src") == src_hash("gemm_tc.cuh" if "gemm" in dom["kernel"] else "norm_fht_quant.cuh"):
+        traffic = rec["bytes"]
+    eff_tops = sum(2.0 * L["spec"].M * L["spec"].N * L["spec"].K for L in layers) / (ms_step / 1e3) / 1e12
+
+    # CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        rows = args.ref_rows
+        dt = oracle_step(oracle_prepare(rows))
+        cpu = {"value": rows / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"first {rows} token rows of each layer, S1-S5 (weights ternarised before timing), "
+                         f"{dt:.1f} s on one host core"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8 codes x ternary, int32 accumulate; fp32 transform",
+        "data": "synthetic (seeded Laplace + outlier channels, bf16)",
+        "config": {"workload": WORKLOAD, "global_batch": M_TOKENS * world, "tokens_per_gpu": M_TOKENS,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (335 MB of bf16 activations per step)"},
+        "effective_tops": eff_tops,
+        "roofline": {"bound": dom["bound"], "achieved": dom["achieved"],
+                     "peak": int8_peak_tops if dom["bound"] == "tensor" else hbm,
+                     "unit": "TOP/s" if dom["bound"] == "tensor" else "GB/s", "frac": dom["frac"],
+                     "traffic": traffic, "kernel": dom["kernel"],
+                     "peak_source": (f"{peak_src} bf16 sustained x2 (int8:bf16 nominal ratio)"
+                                     if dom["bound"] == "tensor" else f"{peak_src} HBM copy")},
+        "kernels": kern,
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk.summary(),
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=64, help="token rows per layer in the CPU-baseline sample")
+    ap.add_argument("--ref-step-rows", type=int, default=1, help="token rows per layer in one reference step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_setup(args.gpus) if args.impl == "ours" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if args.impl == "ours" and world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

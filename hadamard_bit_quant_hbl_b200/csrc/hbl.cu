@@ -1,0 +1,438 @@
+// C ABI of the H-BitLinear forward pass (declared in include/hbl.h): argument checks, kernel
+// selection and launches. All device work is in the kernels included below; the host code
+// only validates, picks a configuration and queues launches on the caller's stream.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "hbl.h"
+
+#include "common.cuh"
+#include "gemm_decode.cuh"
+#include "gemm_tc.cuh"
+#include "norm_fht_quant.cuh"
+#include "pack_weights.cuh"
+
+using namespace hbl;
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+hbl_status cuda_fail(cudaError_t e) {
+  t_last_cuda_error = (int)e;
+  return HBL_ECUDA;
+}
+
+#define HBL_CHECK_LAUNCH()                          \
+  do {                                              \
+    const cudaError_t e_ = cudaGetLastError();      \
+    if (e_ != cudaSuccess) return cuda_fail(e_);    \
+  } while (0)
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline bool is_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+constexpr int kMaxDevices = 64;
+
+int device_sms(int dev) {
+  static int cache[kMaxDevices] = {0};
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  if (cache[dev] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = v > 0 ? v : 148;
+  }
+  return cache[dev];
+}
+
+// Raise a kernel's dynamic shared memory limit when a launch needs more than was allowed so far
+// on the current device (the limit does not change occupancy; the launch's own size does).
+struct SmemLimit {
+  std::mutex mu;
+  int allowed[64] = {0};
+};
+
+template <typename F>
+cudaError_t allow_smem(F* kernel, int bytes, SmemLimit& lim) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  dev &= 63;
+  std::lock_guard<std::mutex> lk(lim.mu);
+  if (lim.allowed[dev] >= bytes) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) lim.allowed[dev] = bytes;
+  return e;
+}
+
+// ---------------------------------------------------------------- packed-weight layout
+
+struct BlobLayout {
+  size_t off0, off1, off2, total;
+};
+
+BlobLayout blob_layout(int K, int N) {
+  BlobLayout b;
+  b.off0 = 0;
+  b.off1 = round_up((size_t)N * K / 4, 256);
+  b.off2 = b.off1 + round_up((size_t)N * K, 256);
+  b.total = b.off2 + round_up((size_t)N * 4, 256);
+  return b;
+}
+
+bool dims_ok(int M, int K) { return M >= 1 && K >= 256 && K <= 32768 && (K % 256) == 0; }
+
+// ---------------------------------------------------------------- fused norm/FHT/quant
+
+template <int L, int EB, int R, bool G>
+hbl_status launch_nfq_t(const NfqArgs& a, int threads, int grid, int smem, cudaStream_t s) {
+  static SmemLimit lim;
+  const cudaError_t e = allow_smem(norm_fht_quant_kernel<L, EB, R, G>, smem, lim);
+  if (e != cudaSuccess) return cuda_fail(e);
+  norm_fht_quant_kernel<L, EB, R, G><<<grid, threads, smem, s>>>(a);
+  HBL_CHECK_LAUNCH();
+  return HBL_OK;
+}
+
+template <int L, int EB, int R>
+hbl_status launch_nfq_g(const NfqArgs& a, int threads, int grid, int smem, cudaStream_t s) {
+  return a.gain ? launch_nfq_t<L, EB, R, true>(a, threads, grid, smem, s)
+                : launch_nfq_t<L, EB, R, false>(a, threads, grid, smem, s);
+}
+
+constexpr int eb_for(int L) {
+  return L == 8 ? 4 : L == 9 ? 5 : L == 10 ? 5 : L == 11 ? 6 : L == 12 ? 6 : 7;
+}
+
+hbl_status run_nfq(const void* X, const float* gain, int M, int K, int had_block, int quant, float eps_norm,
+                   float eps_q, int fmt, void* codes, float* s_x, cudaStream_t stream) {
+  const int n = had_block == 0 ? K : had_block;
+  if (!is_pow2(n) || n < 256 || n > 16384 || (K % n) != 0) return HBL_EUNSUPPORTED;
+  const int L = ilog2_c(n);
+  const int EB = eb_for(L);
+  const int P = 1 << (L - EB);
+  const int nb = K / n;
+  int R = 1, slots = 1, rows = 1;
+  if (nb == 1) {
+    rows = 256 / P;
+    const int cap = (96 * 1024) / (K * 4);
+    if (rows > cap) rows = cap;
+    if (rows < 1) rows = 1;
+    if (P == 16 && rows > 1 && (rows & 1)) rows -= 1;  // half-warp rows come in pairs
+  } else {
+    for (R = 1; R <= 2; ++R) {
+      slots = (nb + R - 1) / R;
+      if (P == 16 && (slots & 1)) ++slots;
+      if (slots * P <= 1024) break;
+    }
+    if (slots * P > 1024) return HBL_EUNSUPPORTED;
+  }
+  const int threads = rows * slots * P;
+  const int smem = rows * K * 4;
+  const int grid = (M + rows - 1) / rows;
+
+  NfqArgs a;
+  a.X = static_cast<const uint16_t*>(X);
+  a.gain = gain;
+  a.codes = static_cast<uint8_t*>(codes);
+  a.s_x = s_x;
+  a.M = M;
+  a.K = K;
+  a.nb = nb;
+  a.quant = quant;
+  a.fmt = fmt;
+  a.eps_norm = eps_norm;
+  a.eps_q = eps_q;
+  a.slots = slots;
+  a.rows = rows;
+
+  switch (L) {
+    case 8: return R == 1 ? launch_nfq_g<8, 4, 1>(a, threads, grid, smem, stream)
+                          : launch_nfq_g<8, 4, 2>(a, threads, grid, smem, stream);
+    case 9: return launch_nfq_g<9, 5, 1>(a, threads, grid, smem, stream);  // nb <= 64 always fits R = 1
+    case 10: return launch_nfq_g<10, 5, 1>(a, threads, grid, smem, stream);
+    case 11: return launch_nfq_g<11, 6, 1>(a, threads, grid, smem, stream);
+    case 12: return launch_nfq_g<12, 6, 1>(a, threads, grid, smem, stream);
+    case 13: return launch_nfq_g<13, 7, 1>(a, threads, grid, smem, stream);
+    case 14: return launch_nfq_g<14, 7, 1>(a, threads, grid, smem, stream);
+    default: return HBL_EUNSUPPORTED;
+  }
+}
+
+// ---------------------------------------------------------------- products
+
+template <int MT, int COLS>
+hbl_status launch_decode_t(const DecodeArgs& a, cudaStream_t s) {
+  const int units = a.K / 64;
+  const int threads = (units + 31) / 32 * 32;
+  const int grid = (a.N + COLS - 1) / COLS;
+  gemm_decode_kernel<MT, COLS><<<grid, threads, 0, s>>>(a);
+  HBL_CHECK_LAUNCH();
+  return HBL_OK;
+}
+
+// Rows are handled MT at a time (one launch per slice of MT rows).
+hbl_status run_decode(const DecodeArgs& a0, cudaStream_t s) {
+  DecodeArgs a = a0;
+  for (a.m0 = 0; a.m0 < a0.M;) {
+    const int left = a0.M - a.m0;
+    hbl_status st;
+    if (left == 1) { st = launch_decode_t<1, 16>(a, s); a.m0 += 1; }
+    else if (left == 2) { st = launch_decode_t<2, 8>(a, s); a.m0 += 2; }
+    else { st = launch_decode_t<4, 4>(a, s); a.m0 += 4; }
+    if (st != HBL_OK) return st;
+  }
+  return HBL_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D K-major int8 operand [rows][K] as a TMA map with a (128 bytes x box_rows) box, 128-byte swizzle.
+bool make_map_i8(CUtensorMap* map, const void* base, int K, int rows, int box_rows) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)K};
+  const cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+hbl_status run_tc(const void* codes_i8, const int8_t* w_i8, const TcArgs& a0, cudaStream_t s) {
+  CUtensorMap mA, mB;
+  if (!make_map_i8(&mA, codes_i8, a0.K, a0.M, kTcBM)) return HBL_ECUDA;
+  if (!make_map_i8(&mB, w_i8, a0.K, a0.N, kTcBN)) return HBL_ECUDA;
+  TcArgs a = a0;
+  a.tiles_m = (a.M + kTcBM - 1) / kTcBM;
+  a.tiles_n = (a.N + kTcBN - 1) / kTcBN;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int ntiles = a.tiles_m * a.tiles_n;
+  const int sms = device_sms(dev);
+  const int grid = ntiles < sms ? ntiles : sms;
+  static SmemLimit lim;
+  const cudaError_t e = allow_smem(gemm_tc_kernel, kTcSmem, lim);
+  if (e != cudaSuccess) return cuda_fail(e);
+  gemm_tc_kernel<<<grid, kTcThreads, kTcSmem, s>>>(mA, mB, a);
+  HBL_CHECK_LAUNCH();
+  return HBL_OK;
+}
+
+// Token counts up to this bound run on CUDA cores over the 2-bit weights.
+constexpr int kDecodeMaxM = 8;
+
+hbl_status run_gemm(const void* codes, int fmt, int abits, const float* s_x, const void* packed, float alpha,
+                    int M, int N, int K, void* Y, int out_dtype, int32_t* acc_debug, cudaStream_t s) {
+  const BlobLayout bl = blob_layout(K, N);
+  const uint8_t* blob = static_cast<const uint8_t*>(packed);
+  const bool packed4 = (abits == 4 && fmt == HBL_CODES_PACKED);
+  if (M <= kDecodeMaxM) {
+    DecodeArgs d;
+    d.m0 = 0;
+    d.codes = static_cast<const uint8_t*>(codes);
+    d.packed4 = packed4 ? 1 : 0;
+    d.s_x = s_x;
+    d.w2 = reinterpret_cast<const uint32_t*>(blob + bl.off0);
+    d.alpha = alpha;
+    d.M = M;
+    d.N = N;
+    d.K = K;
+    d.Y = Y;
+    d.out_bf16 = out_dtype == HBL_OUT_BF16;
+    d.acc_debug = acc_debug;
+    return run_decode(d, s);
+  }
+  if (packed4) return HBL_EUNSUPPORTED;  // the tensor-core path reads one int8 per code
+  TcArgs t;
+  t.s_x = s_x;
+  t.alpha = alpha;
+  t.M = M;
+  t.N = N;
+  t.K = K;
+  t.Y = Y;
+  t.out_bf16 = out_dtype == HBL_OUT_BF16;
+  t.acc_debug = acc_debug;
+  return run_tc(codes, reinterpret_cast<const int8_t*>(blob + bl.off1), t, s);
+}
+
+size_t forward_codes_bytes(int M, int K) { return round_up((size_t)M * K, 256); }
+
+}  // namespace
+
+// =========================================================================== C ABI
+
+extern "C" {
+
+const char* hbl_status_string(hbl_status s) {
+  switch (s) {
+    case HBL_OK: return "HBL_OK";
+    case HBL_EINVAL: return "HBL_EINVAL: invalid argument (null/misaligned pointer, bad size, small buffer)";
+    case HBL_EUNSUPPORTED: return "HBL_EUNSUPPORTED: request outside what the kernels implement";
+    case HBL_ECUDA: return "HBL_ECUDA: a CUDA call failed (see hbl_last_cuda_error)";
+    case HBL_ETIMEOUT: return "HBL_ETIMEOUT: a device-side bounded wait gave up";
+  }
+  return "unknown hbl_status";
+}
+
+int hbl_last_cuda_error(void) { return t_last_cuda_error; }
+
+hbl_status hbl_device_status(hbl_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  int flags = 0;
+  e = cudaMemcpyFromSymbolAsync(&flags, g_error_flags, sizeof(int), 0, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (flags) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbolAsync(g_error_flags, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  if (flags & kErrTimeout) return HBL_ETIMEOUT;
+  if (flags & kErrBadTernary) return HBL_EINVAL;
+  return HBL_OK;
+}
+
+size_t hbl_packed_weights_bytes(int K, int N) {
+  if (K <= 0 || N <= 0) return 0;
+  return blob_layout(K, N).total;
+}
+
+size_t hbl_pack_weights_workspace(int K, int N) {
+  (void)K;
+  (void)N;
+  return round_up((size_t)(kAbsumBlocks + 1) * sizeof(double), 256);
+}
+
+hbl_status hbl_pack_weights(const float* W, int K, int N, float eps_w, void* packed, size_t packed_bytes,
+                            float* alpha_host, void* workspace, size_t ws_bytes, hbl_stream_t stream) {
+  if (!W || !packed || !alpha_host || !workspace) return HBL_EINVAL;
+  if (K < 256 || K > 32768 || (K % 256) || N < 1 || (N % 8)) return HBL_EINVAL;
+  if (!aligned(W, 16) || !aligned(packed, 256) || !aligned(workspace, 16)) return HBL_EINVAL;
+  if (!(eps_w >= 0.f)) return HBL_EINVAL;
+  const BlobLayout bl = blob_layout(K, N);
+  if (packed_bytes < bl.total || ws_bytes < hbl_pack_weights_workspace(K, N)) return HBL_EINVAL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* blob = static_cast<uint8_t*>(packed);
+  double* partials = static_cast<double*>(workspace);
+  double* alpha_d = partials + kAbsumBlocks;
+  cudaError_t e = cudaMemsetAsync(blob + bl.off2, 0, (size_t)N * 4, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const size_t count = (size_t)K * N;
+  absum_partial_kernel<<<kAbsumBlocks, kAbsumThreads, 0, s>>>(W, count / 4, partials);
+  HBL_CHECK_LAUNCH();
+  absum_final_kernel<<<1, kAbsumThreads, 0, s>>>(partials, kAbsumBlocks, (double)count, alpha_d);
+  HBL_CHECK_LAUNCH();
+  dim3 grid((N + 127) / 128, K / 16);
+  ternarize_pack_kernel<false><<<grid, 128, 0, s>>>(W, nullptr, K, N, alpha_d, (double)eps_w,
+                                                     reinterpret_cast<uint32_t*>(blob + bl.off0),
+                                                     reinterpret_cast<int8_t*>(blob + bl.off1),
+                                                     reinterpret_cast<int32_t*>(blob + bl.off2));
+  HBL_CHECK_LAUNCH();
+  double alpha = 0.0;
+  e = cudaMemcpyAsync(&alpha, alpha_d, sizeof(double), cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  *alpha_host = (float)alpha;
+  return HBL_OK;
+}
+
+hbl_status hbl_pack_ternary(const int8_t* t, int K, int N, void* packed, size_t packed_bytes,
+                            hbl_stream_t stream) {
+  if (!t || !packed) return HBL_EINVAL;
+  if (K < 256 || K > 32768 || (K % 256) || N < 1 || (N % 8)) return HBL_EINVAL;
+  if (!aligned(packed, 256)) return HBL_EINVAL;
+  const BlobLayout bl = blob_layout(K, N);
+  if (packed_bytes < bl.total) return HBL_EINVAL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* blob = static_cast<uint8_t*>(packed);
+  cudaError_t e = cudaMemsetAsync(blob + bl.off2, 0, (size_t)N * 4, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  dim3 grid((N + 127) / 128, K / 16);
+  ternarize_pack_kernel<true><<<grid, 128, 0, s>>>(nullptr, t, K, N, nullptr, 0.0,
+                                                    reinterpret_cast<uint32_t*>(blob + bl.off0),
+                                                    reinterpret_cast<int8_t*>(blob + bl.off1),
+                                                    reinterpret_cast<int32_t*>(blob + bl.off2));
+  HBL_CHECK_LAUNCH();
+  return HBL_OK;
+}
+
+hbl_status hbl_norm_fht_quant(const void* X, const float* gain, int M, int K, int had_block, hbl_quant quant,
+                              float eps_norm, float eps_q, hbl_codes_fmt fmt, void* codes, float* s_x,
+                              hbl_stream_t stream) {
+  if (!X || !codes || !s_x) return HBL_EINVAL;
+  if (!dims_ok(M, K)) return HBL_EINVAL;
+  if (!aligned(X, 16) || !aligned(codes, 16) || !aligned(s_x, 4) || (gain && !aligned(gain, 4)))
+    return HBL_EINVAL;
+  if (quant != HBL_Q_A8_ABSMAX && quant != HBL_Q_A4_ABSMEAN && quant != HBL_Q_A4_ABSMAX) return HBL_EUNSUPPORTED;
+  if (fmt != HBL_CODES_PACKED && fmt != HBL_CODES_I8) return HBL_EINVAL;
+  if (!(eps_norm >= 0.f) || !(eps_q >= 0.f)) return HBL_EINVAL;
+  if (had_block < 0) return HBL_EINVAL;
+  return run_nfq(X, gain, M, K, had_block, (int)quant, eps_norm, eps_q, (int)fmt, codes, s_x,
+                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+hbl_status hbl_ternary_gemm(const void* codes, hbl_codes_fmt fmt, int abits, const float* s_x, const void* packed,
+                            size_t packed_bytes, float alpha, int M, int N, int K, void* Y, hbl_out_dtype out_dtype,
+                            int32_t* acc_debug, hbl_stream_t stream) {
+  if (!codes || !s_x || !packed || !Y) return HBL_EINVAL;
+  if (!dims_ok(M, K) || N < 8 || (N % 8)) return HBL_EINVAL;
+  if (abits != 4 && abits != 8) return HBL_EUNSUPPORTED;
+  if (fmt != HBL_CODES_PACKED && fmt != HBL_CODES_I8) return HBL_EINVAL;
+  if (out_dtype != HBL_OUT_F32 && out_dtype != HBL_OUT_BF16) return HBL_EINVAL;
+  if (!aligned(codes, 16) || !aligned(packed, 256) || !aligned(Y, 16) || !aligned(s_x, 4) ||
+      (acc_debug && !aligned(acc_debug, 4)))
+    return HBL_EINVAL;
+  if (packed_bytes < blob_layout(K, N).total) return HBL_EINVAL;
+  return run_gemm(codes, (int)fmt, abits, s_x, packed, alpha, M, N, K, Y, (int)out_dtype, acc_debug,
+                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t hbl_forward_workspace(int M, int K, hbl_quant quant) {
+  (void)quant;
+  if (M <= 0 || K <= 0) return 0;
+  return forward_codes_bytes(M, K) + round_up((size_t)M * 4, 256);
+}
+
+hbl_status hbl_forward(const void* X, const float* gain, const void* packed, size_t packed_bytes, float alpha, int M,
+                       int K, int N, int had_block, hbl_quant quant, float eps_norm, float eps_q, void* workspace,
+                       size_t ws_bytes, void* Y, hbl_out_dtype out_dtype, hbl_stream_t stream) {
+  if (!X || !packed || !workspace || !Y) return HBL_EINVAL;
+  if (!dims_ok(M, K) || N < 8 || (N % 8)) return HBL_EINVAL;
+  if (!aligned(workspace, 256)) return HBL_EINVAL;
+  if (ws_bytes < hbl_forward_workspace(M, K, quant)) return HBL_EINVAL;
+  if (packed_bytes < blob_layout(K, N).total || !aligned(packed, 256) || !aligned(Y, 16)) return HBL_EINVAL;
+  const int abits = quant == HBL_Q_A8_ABSMAX ? 8 : 4;
+  const hbl_codes_fmt fmt = M <= kDecodeMaxM ? HBL_CODES_PACKED : HBL_CODES_I8;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* codes = ws;
+  float* s_x = reinterpret_cast<float*>(ws + forward_codes_bytes(M, K));
+  hbl_status st = hbl_norm_fht_quant(X, gain, M, K, had_block, quant, eps_norm, eps_q, fmt, codes, s_x, stream);
+  if (st != HBL_OK) return st;
+  return hbl_ternary_gemm(codes, fmt, abits, s_x, packed, packed_bytes, alpha, M, N, K, Y, out_dtype, nullptr,
+                          stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,114 @@
+// Offline weight preparation: per-tensor absmean ternarisation and packing.
+//
+// Method: BitNet v2 walkthrough article (m.jxzklqfsx.com), section "H-BitLinear模塊" (weights
+// ternarised to {-1, 0, 1} with a per-tensor absmean scale) and the bitnet.cpp news article
+// (gubiw.cn), section "6 页论文，引入 1 bit LLM" (divide the weight matrix by its mean
+// absolute value, round each entry to the nearest of -1, 0, 1).
+//
+// alpha is reduced in fp64 in a fixed order (per-block partial sums, then one block sums the
+// partials), so the result does not depend on scheduling. The rounding decision
+// rint(W / (alpha + eps)) is also taken in fp64.
+#pragma once
+
+#include "common.cuh"
+
+namespace hbl {
+
+constexpr int kAbsumBlocks = 4 * 148;
+constexpr int kAbsumThreads = 256;
+
+// Fixed-order tree reduction of one double per thread of a 256-thread block.
+__device__ __forceinline__ double block_sum_256(double v, double* sh) {
+  sh[threadIdx.x] = v;
+  __syncthreads();
+#pragma unroll
+  for (int s = 128; s > 0; s >>= 1) {
+    if (threadIdx.x < s) sh[threadIdx.x] += sh[threadIdx.x + s];
+    __syncthreads();
+  }
+  return sh[0];
+}
+
+__global__ void __launch_bounds__(kAbsumThreads) absum_partial_kernel(const float* __restrict__ W,
+                                                                      size_t count4,
+                                                                      double* __restrict__ partials) {
+  __shared__ double sh[kAbsumThreads];
+  double acc = 0.0;
+  const float4* W4 = reinterpret_cast<const float4*>(W);
+  for (size_t i = (size_t)blockIdx.x * kAbsumThreads + threadIdx.x; i < count4;
+       i += (size_t)gridDim.x * kAbsumThreads) {
+    const float4 w = __ldg(W4 + i);
+    acc += (double)fabsf(w.x) + (double)fabsf(w.y) + (double)fabsf(w.z) + (double)fabsf(w.w);
+  }
+  const double s = block_sum_256(acc, sh);
+  if (threadIdx.x == 0) partials[blockIdx.x] = s;
+}
+
+__global__ void __launch_bounds__(kAbsumThreads) absum_final_kernel(const double* __restrict__ partials,
+                                                                    int nparts, double count,
+                                                                    double* __restrict__ alpha_out) {
+  __shared__ double sh[kAbsumThreads];
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < nparts; i += kAbsumThreads) acc += partials[i];
+  const double s = block_sum_256(acc, sh);
+  if (threadIdx.x == 0) alpha_out[0] = s / count;
+}
+
+// One thread per (column n, 16-row group w): 16 ternary codes t[16w .. 16w+15][n].
+// Lanes take consecutive n, so every read of a W row segment is coalesced.
+//   section 0: uint32 word (n, w), code t+1 of k = 16w + 4s + b at bits 8b + 2s
+//   section 1: int8 t[k][n] at n*K + k
+//   section 2: int32 column sum (atomic, integer: order-independent)
+template <bool FROM_CODES>
+__global__ void __launch_bounds__(128) ternarize_pack_kernel(const float* __restrict__ W,
+                                                             const int8_t* __restrict__ T, int K, int N,
+                                                             const double* __restrict__ alpha_d,
+                                                             double eps_w, uint32_t* __restrict__ sec0,
+                                                             int8_t* __restrict__ sec1,
+                                                             int32_t* __restrict__ sec2) {
+  const int n = blockIdx.x * 128 + threadIdx.x;
+  const int w = blockIdx.y;
+  if (n >= N) return;
+  int t[16];
+  if constexpr (FROM_CODES) {
+    bool bad = false;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      int v = T[(size_t)(16 * w + j) * N + n];
+      if (v < -1 || v > 1) {
+        bad = true;
+        v = v < -1 ? -1 : 1;
+      }
+      t[j] = v;
+    }
+    if (bad) raise_error(kErrBadTernary);
+  } else {
+    const double denom = alpha_d[0] + eps_w;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const double x = (double)W[(size_t)(16 * w + j) * N + n];
+      double q = denom > 0.0 ? rint(x / denom) : 0.0;
+      q = q < -1.0 ? -1.0 : (q > 1.0 ? 1.0 : q);
+      t[j] = (int)q;
+    }
+  }
+  uint32_t word = 0;
+  int colsum = 0;
+  uint32_t b4[4];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int s = j >> 2, b = j & 3;  // k = 16w + 4s + b
+    word |= (uint32_t)(t[j] + 1) << (8 * b + 2 * s);
+    colsum += t[j];
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    b4[q] = ((uint32_t)(uint8_t)(int8_t)t[4 * q]) | ((uint32_t)(uint8_t)(int8_t)t[4 * q + 1] << 8) |
+            ((uint32_t)(uint8_t)(int8_t)t[4 * q + 2] << 16) | ((uint32_t)(uint8_t)(int8_t)t[4 * q + 3] << 24);
+  }
+  sec0[(size_t)n * (K / 16) + w] = word;
+  *reinterpret_cast<uint4*>(sec1 + (size_t)n * K + 16 * w) = make_uint4(b4[0], b4[1], b4[2], b4[3]);
+  atomicAdd(sec2 + n, colsum);
+}
+
+}  // namespace hbl

@@ -1,0 +1,174 @@
+/*
+ * hbl.h -- C ABI of the H-BitLinear forward pass (BitNet v2) for NVIDIA B200 (sm_100a).
+ *
+ * The layer, as stated in "BitNet v2: Native 4-bit Activations with Hadamard
+ * Transformation for 1-bit LLMs" (abstract) and in the Chinese walkthrough of that
+ * paper (m.jxzklqfsx.com, section "H-BitLinear模塊"):
+ *
+ *     Y = Q_w(W) . Q_a( Hadamard( RMSNorm(X) ) )
+ *
+ *   Q_w  per-tensor absmean ternarisation of the weights to {-1, 0, +1} with scale alpha
+ *   Hadamard  online fast Walsh-Hadamard transform along the K features of each token
+ *   Q_a  per-token activation quantisation to INT8 (absmax) or INT4 (absmean or absmax)
+ *
+ * Conventions shared by every call
+ *   - Every pointer argument is a DEVICE pointer owned by the caller, unless its
+ *     name ends in _host. The library never allocates or frees memory.
+ *   - Every call is stream-ordered on `stream` (0 = legacy default stream) and
+ *     returns as soon as its kernels are queued, except hbl_pack_weights, which
+ *     synchronises `stream` to hand alpha back to the host.
+ *   - Matrices are row-major and densely packed (row stride = row length).
+ *   - No call keeps state between calls; all of them are thread-safe as long as
+ *     two concurrent calls do not write the same buffers.
+ *   - Errors are returned as hbl_status; nothing is thrown across the ABI. On
+ *     HBL_ECUDA, hbl_last_cuda_error() (thread-local) gives the CUDA error code.
+ *     Device-side bounded waits that give up are reported by the next
+ *     hbl_device_status() call as HBL_ETIMEOUT.
+ *
+ * Scalar sizes: 1 <= M, 1 <= N, K a multiple of 256, K <= 32768.
+ */
+#ifndef HBL_H_
+#define HBL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* hbl_stream_t; /* same type as cudaStream_t */
+
+typedef enum hbl_status {
+  HBL_OK = 0,
+  HBL_EINVAL = 1,        /* null or misaligned pointer, bad size, buffer too small */
+  HBL_EUNSUPPORTED = 2,  /* valid request outside what the kernels implement */
+  HBL_ECUDA = 3,         /* a CUDA call failed; see hbl_last_cuda_error() */
+  HBL_ETIMEOUT = 4       /* a device-side bounded wait gave up (kernel returned early) */
+} hbl_status;
+
+/* Activation quantiser (per token row). */
+typedef enum hbl_quant {
+  HBL_Q_A8_ABSMAX = 0,  /* gamma = max|x|,  q = RoundClip(127 x/(gamma+eps), -128, 127), s = gamma/127 */
+  HBL_Q_A4_ABSMEAN = 1, /* beta  = mean|x|, q = RoundClip(sqrt7 x/(beta+eps), -8, 7),    s = beta/sqrt7 */
+  HBL_Q_A4_ABSMAX = 2   /* gamma = max|x|,  q = RoundClip(7 x/(gamma+eps), -8, 7),        s = gamma/7   */
+} hbl_quant;
+
+/* Layout of activation codes [M][K]. */
+typedef enum hbl_codes_fmt {
+  HBL_CODES_PACKED = 0, /* a4: two int4 two's-complement codes per byte, element 2j in the low
+                           nibble of byte j of the row (row = K/2 bytes); a8: one int8 per element */
+  HBL_CODES_I8 = 1      /* one int8 per element for a4 as well (row = K bytes) */
+} hbl_codes_fmt;
+
+typedef enum hbl_out_dtype { HBL_OUT_F32 = 0, HBL_OUT_BF16 = 1 } hbl_out_dtype;
+
+/* Human-readable name of a status code (static string). */
+const char* hbl_status_string(hbl_status s);
+
+/* CUDA error code (cudaError_t) of the last HBL_ECUDA on the calling thread. */
+int hbl_last_cuda_error(void);
+
+/* Reads and clears the device-side error flag of the current device. Synchronises `stream`.
+ * Returns HBL_ETIMEOUT if any kernel of this library gave up a bounded wait since the last
+ * call, HBL_OK otherwise (or HBL_ECUDA if the synchronisation itself failed). */
+hbl_status hbl_device_status(hbl_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Packed ternary weights.
+ *
+ * Weight ternarisation follows the walkthrough article, section "H-BitLinear模塊" (per-tensor
+ * absmean ternarisation to {-1,0,1}), and the bitnet.cpp news article, section
+ * "6 页论文，引入 1 bit LLM" (scale by the mean absolute value, round to the nearest of
+ * -1, 0, 1):  alpha = mean|W| over all K*N entries; t = RoundClip(W/(alpha+eps_w), -1, 1).
+ *
+ * The packed blob (hbl_packed_weights_bytes(K, N) bytes, 256-byte aligned) holds, for the
+ * logical K x N ternary matrix t:
+ *   section 0 at byte 0:   2-bit codes, N rows of K/16 uint32 words (K-major). Word w of
+ *                          row n holds t[16w + 4s + b][n] + 1 (in {0,1,2}) at bits 8b+2s
+ *                          (b, s in 0..3). Read by the small-M (decode) product.
+ *   section 1 at byte A1:  int8 t[k][n] as N rows of K bytes (K-major). Read by the
+ *                          tensor-core product.
+ *   section 2 at byte A2:  int32 column sums sum_k t[k][n], N entries.
+ *   with A1 = round_up(N*K/4, 256), A2 = A1 + round_up(N*K, 256).
+ * ------------------------------------------------------------------------------------- */
+size_t hbl_packed_weights_bytes(int K, int N);
+
+/* Scratch needed by hbl_pack_weights (bytes). */
+size_t hbl_pack_weights_workspace(int K, int N);
+
+/* Ternarise fp32 W [K][N] (row-major) into `packed` and return alpha.
+ *   W          device, K*N floats, 4-byte aligned
+ *   eps_w      added to alpha in the divisor (0 = plain absmean; an all-zero W gives t = 0)
+ *   packed     device, packed_bytes >= hbl_packed_weights_bytes(K, N), 256-byte aligned
+ *   alpha_host HOST pointer: receives alpha as float (also the device value rounded to float)
+ *   workspace  device scratch of ws_bytes >= hbl_pack_weights_workspace(K, N), 16-byte aligned
+ * Synchronises `stream` before returning (alpha is read back). */
+hbl_status hbl_pack_weights(const float* W, int K, int N, float eps_w, void* packed,
+                            size_t packed_bytes, float* alpha_host, void* workspace,
+                            size_t ws_bytes, hbl_stream_t stream);
+
+/* Pack given ternary codes t [K][N] (int8 in {-1,0,1}, row-major) into `packed`.
+ * Entries outside {-1,0,1} give HBL_EINVAL only through hbl_device_status (they are
+ * clamped and flagged, not trapped). Asynchronous. */
+hbl_status hbl_pack_ternary(const int8_t* t, int K, int N, void* packed, size_t packed_bytes,
+                            hbl_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Activation side: RMSNorm -> Hadamard -> per-token quantisation, fused in one kernel.
+ *
+ *   r      = sqrt(mean_k x[m,k]^2 + eps_norm)                  (RMSNorm; LLaMA-like parts, article
+ *   xhat   = x / r * gain  (gain may be NULL = all ones)        section "BitNet v2：原生4位激活")
+ *   xr     = H xhat, H = Sylvester Walsh-Hadamard / sqrt(n)     (fast transform in O(n log n),
+ *            applied to all of K when had_block = 0 (K must    article section "H-BitLinear模塊")
+ *            be a power of two), or to each consecutive block
+ *            of had_block features (block-diagonal)
+ *   q, s   = quantiser `quant` applied per token row (see hbl_quant); a row whose statistic
+ *            is 0 gives q = 0, s = 0. Rounding: nearest, ties to even, decided in fp32.
+ *
+ *   X       device bf16 [M][K], 16-byte aligned
+ *   gain    device fp32 [K] or NULL
+ *   had_block 0, or a power of two in [256, 16384] dividing K; when 0, K must be a power of two
+ *           in [256, 16384]
+ *   codes   device, M rows in `fmt` (see hbl_codes_fmt), 16-byte aligned
+ *   s_x     device fp32 [M]
+ * Asynchronous. */
+hbl_status hbl_norm_fht_quant(const void* X, const float* gain, int M, int K, int had_block,
+                              hbl_quant quant, float eps_norm, float eps_q, hbl_codes_fmt fmt,
+                              void* codes, float* s_x, hbl_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Ternary x low-bit product with dequant epilogue:
+ *
+ *   Y[m,n] = s_x[m] * alpha * sum_k q[m,k] * t[k,n]
+ *
+ * (the layer's product Q_w(W) . Q_a(...) with both scales applied after the integer sum).
+ *   codes, fmt, abits  activation codes as written by hbl_norm_fht_quant (abits 4 or 8)
+ *   s_x      device fp32 [M]
+ *   packed   blob from hbl_pack_weights / hbl_pack_ternary for this K, N
+ *   Y        device [M][N] of out_dtype (fp32 or bf16), 16-byte aligned, N a multiple of 8
+ *   acc_debug  device int32 [M][N] receiving the exact integer sums, or NULL
+ * Small M runs on CUDA cores over the 2-bit section; large M on tcgen05 int8 tensor cores
+ * over the int8 section (which then needs fmt = HBL_CODES_I8 or abits = 8).
+ * Asynchronous. */
+hbl_status hbl_ternary_gemm(const void* codes, hbl_codes_fmt fmt, int abits, const float* s_x,
+                            const void* packed, size_t packed_bytes, float alpha, int M, int N,
+                            int K, void* Y, hbl_out_dtype out_dtype, int32_t* acc_debug,
+                            hbl_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * The whole layer forward: hbl_norm_fht_quant into `workspace`, then hbl_ternary_gemm.
+ *   workspace  device scratch, ws_bytes >= hbl_forward_workspace(M, K, quant), 256-byte aligned
+ * Asynchronous. */
+size_t hbl_forward_workspace(int M, int K, hbl_quant quant);
+
+hbl_status hbl_forward(const void* X, const float* gain, const void* packed, size_t packed_bytes,
+                       float alpha, int M, int K, int N, int had_block, hbl_quant quant,
+                       float eps_norm, float eps_q, void* workspace, size_t ws_bytes, void* Y,
+                       hbl_out_dtype out_dtype, hbl_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HBL_H_ */

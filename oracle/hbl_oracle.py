@@ -203,8 +203,8 @@ def norm_fht_quant(x: np.ndarray, gain: np.ndarray | None, had_block: int, abits
 
 
 def ternary_matmul(q: np.ndarray, t: np.ndarray) -> np.ndarray:
-    """acc[m, n] = sum_k q[m, k] * t[k, n] in exact int64 arithmetic."""
-    return np.asarray(q, dtype=np.int64) @ np.asarray(t, dtype=np.int64)
+    """acc[m, n] = sum_k q[m, k] * t[k, n] in exact int64 arithmetic (the sum written as an einsum)."""
+    return np.einsum("mk,kn->mn", np.asarray(q, dtype=np.int64), np.asarray(t, dtype=np.int64))
 
 
 def dequant(acc: np.ndarray, s: np.ndarray, alpha: float) -> np.ndarray:

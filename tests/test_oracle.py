@@ -193,6 +193,8 @@ def test_ternary_matmul_brute_force_and_blas():
     t = RNG.integers(-1, 2, size=(4096, 48)).astype(np.int8)
     np.testing.assert_array_equal(oracle.ternary_matmul(q, t),
                                   (q.astype(np.float64) @ t.astype(np.float64)).astype(np.int64))
+    # and numpy's integer matmul (a third routine)
+    np.testing.assert_array_equal(oracle.ternary_matmul(q, t), q.astype(np.int64) @ t.astype(np.int64))
 
 
 # ---------------------------------------------------------------- worked example
