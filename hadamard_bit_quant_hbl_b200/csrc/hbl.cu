@@ -88,20 +88,40 @@ bool dims_ok(int M, int K) { return M >= 1 && K >= 256 && K <= 32768 && (K % 256
 
 // ---------------------------------------------------------------- fused norm/FHT/quant
 
-template <int L, int EB, int R, bool G>
-hbl_status launch_nfq_t(const NfqArgs& a, int threads, int grid, int smem, cudaStream_t s) {
+// Persistent grid: as many CTAs as fit on the device at once (at most one per row group).
+template <typename F>
+int persistent_grid(F* kernel, int threads, int smem, int groups) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  const int g = device_sms(dev) * per_sm;
+  return groups < g ? groups : g;
+}
+
+template <int L, int EB, int R, bool G, int QM>
+hbl_status launch_nfq_t(const NfqArgs& a, int threads, int smem, cudaStream_t s) {
   static SmemLimit lim;
-  const cudaError_t e = allow_smem(norm_fht_quant_kernel<L, EB, R, G>, smem, lim);
+  auto* k = norm_fht_quant_kernel<L, EB, R, G, QM>;
+  const cudaError_t e = allow_smem(k, smem, lim);
   if (e != cudaSuccess) return cuda_fail(e);
-  norm_fht_quant_kernel<L, EB, R, G><<<grid, threads, smem, s>>>(a);
+  const int grid = persistent_grid(k, threads, smem, a.groups);
+  k<<<grid, threads, smem, s>>>(a);
   HBL_CHECK_LAUNCH();
   return HBL_OK;
 }
 
 template <int L, int EB, int R>
-hbl_status launch_nfq_g(const NfqArgs& a, int threads, int grid, int smem, cudaStream_t s) {
-  return a.gain ? launch_nfq_t<L, EB, R, true>(a, threads, grid, smem, s)
-                : launch_nfq_t<L, EB, R, false>(a, threads, grid, smem, s);
+hbl_status launch_nfq_g(const NfqArgs& a, int quant, int threads, int smem, cudaStream_t s) {
+  if (a.gain) {
+    if (quant == 0) return launch_nfq_t<L, EB, R, true, 0>(a, threads, smem, s);
+    if (quant == 1) return launch_nfq_t<L, EB, R, true, 1>(a, threads, smem, s);
+    return launch_nfq_t<L, EB, R, true, 2>(a, threads, smem, s);
+  }
+  if (quant == 0) return launch_nfq_t<L, EB, R, false, 0>(a, threads, smem, s);
+  if (quant == 1) return launch_nfq_t<L, EB, R, false, 1>(a, threads, smem, s);
+  return launch_nfq_t<L, EB, R, false, 2>(a, threads, smem, s);
 }
 
 constexpr int eb_for(int L) {
@@ -118,22 +138,26 @@ hbl_status run_nfq(const void* X, const float* gain, int M, int K, int had_block
   const int nb = K / n;
   int R = 1, slots = 1, rows = 1;
   if (nb == 1) {
+    // a group of rows per CTA: about 256 threads and <= 96 KB of shared memory (bf16 landing
+    // buffer + fp32 regrouping buffer), so that two CTAs fit on an SM
     rows = 256 / P;
-    const int cap = (96 * 1024) / (K * 4);
+    const int cap = (96 * 1024) / (K * 6);
     if (rows > cap) rows = cap;
     if (rows < 1) rows = 1;
     if (P == 16 && rows > 1 && (rows & 1)) rows -= 1;  // half-warp rows come in pairs
   } else {
-    for (R = 1; R <= 2; ++R) {
+    // one row per CTA; each thread transforms R blocks in turn so that the CTA stays within the
+    // plan's thread bound
+    const int maxt = nfq_max_threads(L);
+    for (R = 1; R <= 4; R *= 2) {
       slots = (nb + R - 1) / R;
       if (P == 16 && (slots & 1)) ++slots;
-      if (slots * P <= 1024) break;
+      if (slots * P <= maxt) break;
     }
-    if (slots * P > 1024) return HBL_EUNSUPPORTED;
+    if (slots * P > maxt) return HBL_EUNSUPPORTED;
   }
   const int threads = rows * slots * P;
-  const int smem = rows * K * 4;
-  const int grid = (M + rows - 1) / rows;
+  const int smem = rows * K * 6;
 
   NfqArgs a;
   a.X = static_cast<const uint16_t*>(X);
@@ -143,22 +167,29 @@ hbl_status run_nfq(const void* X, const float* gain, int M, int K, int had_block
   a.M = M;
   a.K = K;
   a.nb = nb;
-  a.quant = quant;
   a.fmt = fmt;
   a.eps_norm = eps_norm;
   a.eps_q = eps_q;
   a.slots = slots;
   a.rows = rows;
+  a.groups = (M + rows - 1) / rows;
 
+  // K <= 32768 bounds nb, so these R always suffice: L=8 nb<=128 (R<=4), L=9..12 R<=2, L>=13 R=1
   switch (L) {
-    case 8: return R == 1 ? launch_nfq_g<8, 4, 1>(a, threads, grid, smem, stream)
-                          : launch_nfq_g<8, 4, 2>(a, threads, grid, smem, stream);
-    case 9: return launch_nfq_g<9, 5, 1>(a, threads, grid, smem, stream);  // nb <= 64 always fits R = 1
-    case 10: return launch_nfq_g<10, 5, 1>(a, threads, grid, smem, stream);
-    case 11: return launch_nfq_g<11, 6, 1>(a, threads, grid, smem, stream);
-    case 12: return launch_nfq_g<12, 6, 1>(a, threads, grid, smem, stream);
-    case 13: return launch_nfq_g<13, 7, 1>(a, threads, grid, smem, stream);
-    case 14: return launch_nfq_g<14, 7, 1>(a, threads, grid, smem, stream);
+    case 8:
+      if (R == 1) return launch_nfq_g<8, 4, 1>(a, quant, threads, smem, stream);
+      if (R == 2) return launch_nfq_g<8, 4, 2>(a, quant, threads, smem, stream);
+      return launch_nfq_g<8, 4, 4>(a, quant, threads, smem, stream);
+    case 9: return R == 1 ? launch_nfq_g<9, 5, 1>(a, quant, threads, smem, stream)
+                          : launch_nfq_g<9, 5, 2>(a, quant, threads, smem, stream);
+    case 10: return R == 1 ? launch_nfq_g<10, 5, 1>(a, quant, threads, smem, stream)
+                           : launch_nfq_g<10, 5, 2>(a, quant, threads, smem, stream);
+    case 11: return R == 1 ? launch_nfq_g<11, 6, 1>(a, quant, threads, smem, stream)
+                           : launch_nfq_g<11, 6, 2>(a, quant, threads, smem, stream);
+    case 12: return R == 1 ? launch_nfq_g<12, 6, 1>(a, quant, threads, smem, stream)
+                           : launch_nfq_g<12, 6, 2>(a, quant, threads, smem, stream);
+    case 13: return launch_nfq_g<13, 7, 1>(a, quant, threads, smem, stream);
+    case 14: return launch_nfq_g<14, 7, 1>(a, quant, threads, smem, stream);
     default: return HBL_EUNSUPPORTED;
   }
 }

@@ -4,21 +4,27 @@
 // applies an online Hadamard transform, computed with the fast Hadamard transform in
 // O(n log n), to the normalised activations before quantising them per token to INT8 or INT4.
 //
-// Data flow of one token row (K = nb blocks of n = 2^L features; nb = 1 for a full transform):
-//   1. 16-byte coalesced bf16 loads straight into registers ("layout 1"): a thread holds
-//      E = 2^EB values of a block: 8 consecutive features (index bits 0..2) for each of the
-//      2^(EB-3) top index bits. Sum of squares for the RMS accumulates here.
-//   2. All EB butterfly stages whose index bits live in registers run in registers.
-//   3. One pass through shared memory (XOR-swizzled so that both the write and the read are
-//      free of bank conflicts) regroups the values so that the remaining L-EB index bits live
-//      in registers ("layout 2"); their butterfly stages run in registers.
-//   4. The row statistic (max|y| or sum|y|) and the sum of squares are reduced across the
-//      threads of the row; the codes are decided in fp32 and written as bytes to shared memory
-//      (second XOR swizzle), then streamed out with 16-byte loads and 8/16-byte stores.
-// The butterflies act on the raw x (times gain); the RMS factor and the 1/sqrt(n) of the
-// orthonormal transform only rescale the row, so they are folded into the per-row multiplier
-// and into s_x. Stage order differs from a textbook loop; in exact arithmetic the stages
-// commute, in fp32 the result differs by rounding only.
+// The kernel is persistent: a CTA owns a group of `rows` token rows at a time and walks over
+// the groups; while it transforms one group, the TMA engine copies the next group's bf16 rows
+// into shared memory (one 1-D bulk copy, completion on an mbarrier).
+//
+// One token row has K = nb blocks of n = 2^L features (nb = 1 for a transform over all of K).
+// A block is transformed by P = 2^(L-EB) threads holding E = 2^EB values each:
+//   1. "layout 1": a thread holds 8 consecutive features (index bits 0..2) for each of the
+//      2^(EB-3) top index bits; read from the landing buffer as 16-byte vectors; the sum of
+//      squares for the RMS accumulates here; all EB butterfly stages run in registers.
+//   2. one pass through shared memory (128-bit stores, scalar loads, XOR swizzle checked at
+//      compile time) regroups the values so that index bits 3..TOP-1 are in registers
+//      ("layout 2"); their L-EB butterfly stages run in registers.
+//   3. the row statistic (max|y| or sum|y|) and the sum of squares are reduced over the row;
+//      codes are decided in fp32 (product with the per-row multiplier, then round to nearest
+//      even), written to a byte matrix [k mod 8][k / 8] in shared memory with 128-bit stores,
+//      and streamed out in natural order after a register byte transpose.
+// Butterflies use packed fp32x2 adds (two butterflies per instruction) except on the register
+// bit that pairs the two halves of a float2. They act on the raw x (times gain): the RMS factor
+// and the 1/sqrt(n) of the orthonormal transform only rescale the row, so they are folded into
+// the per-row multiplier and into s_x. The stage order differs from a textbook loop; in exact
+// arithmetic the stages commute, in fp32 the result differs by rounding only.
 #pragma once
 
 #include "common.cuh"
@@ -31,11 +37,11 @@ struct NfqArgs {
   uint8_t* codes;
   float* s_x;
   int M, K, nb;       // nb = K / n
-  int quant;          // hbl_quant
   int fmt;            // hbl_codes_fmt
   float eps_norm, eps_q;
   int slots;          // blocks of a row transformed concurrently (threads per row = slots * P)
-  int rows;           // token rows per CTA
+  int rows;           // token rows per group
+  int groups;         // ceil(M / rows)
 };
 
 // ---------------------------------------------------------------- compile-time plan
@@ -46,13 +52,14 @@ struct FhtPlan {
   static constexpr int n = 1 << L;
   static constexpr int P = 1 << (L - EB);    // threads per block transform
   static constexpr int E = 1 << EB;          // values per thread per block
-  static constexpr int NV = 1 << (EB - 3);   // 16-byte vectors per thread per block (layout 1)
+  static constexpr int NV = 1 << (EB - 3);   // 8-feature vectors per thread per block (layout 1)
   static constexpr int TOP = L - (EB - 3);   // lowest index bit of the register "top" bits
   static constexpr int XB = 2 * EB - L;      // index bits 0..XB-1 also held in registers in layout 2
   static constexpr int S2 = L - EB;          // butterfly stages run in layout 2
-  static_assert(EB >= 3 && XB >= 0 && XB <= 3, "unsupported transform split");
+  static_assert(EB >= 3 && XB >= 0 && XB <= 1, "unsupported transform split");
+  static_assert(S2 >= 4, "layout 2 writes codes in 16-byte groups");
   static_assert(P == 16 || P % 32 == 0, "threads per block must be 16 or a multiple of 32");
-  static_assert(TOP >= 7, "byte swizzle needs TOP >= 7");
+  static_assert(TOP >= 7, "swizzle needs TOP >= 7");
 
   // Layout 1: register r = (vv << 3) | e, thread p  ->  index (vv << TOP) | (p << 3) | e
   static __host__ __device__ constexpr int idx1(int p, int r) {
@@ -64,150 +71,98 @@ struct FhtPlan {
     return ((r & ((1 << S2) - 1)) << 3) | (r >> S2) | ((p & ((1 << (3 - XB)) - 1)) << XB) |
            ((p >> (3 - XB)) << TOP);
   }
-
-  // Address bits that vary across the 32 lanes of a warp in each layout. When P == 16 the
-  // fifth lane bit selects the neighbouring block (or row), i.e. address bit L.
-  static constexpr uint32_t lanes1() {
-    uint32_t m = 0;
-    for (int b = 0; b < 5; ++b) {
-      if ((1 << b) < P) m |= (uint32_t)idx1(1 << b, 0);
-      else m |= 1u << L;
-    }
-    return m;
-  }
-  static constexpr uint32_t lanes2() {
-    uint32_t m = 0;
-    for (int b = 0; b < 5; ++b) {
-      if ((1 << b) < P) m |= (uint32_t)idx2(1 << b, 0);
-      else m |= 1u << L;
-    }
-    return m;
-  }
-
-  // Byte swizzle of the code staging buffer: XOR byte-address bits 3..6 with bits TOP..TOP+3.
-  static __host__ __device__ constexpr uint32_t bswz(uint32_t a) {
-    return a ^ (((a >> TOP) & 15u) << 3);
-  }
-};
-
-
-// Float swizzle of the regrouping buffer for a plan: bank bit k (address bit k, k < 5) is XORed
-// with the parity of (a & S[k]), where S[k] only holds address bits >= 5 (so the map is a
-// bijection on every 32-word row). Each layout's lane bits >= 5 are assigned to the bank bits
-// that this layout's own low lane bits do not already drive; a lane bit shared by both layouts
-// drives one free bank bit of each. check_layout() verifies exhaustively, at compile time, that
-// every warp access of both layouts is free of bank conflicts.
-template <class Pl>
-struct FhtSwizzle {
-  struct Masks {
-    uint32_t S[5];
-  };
-  static constexpr Masks solve() {
-    Masks s{{0, 0, 0, 0, 0}};
-    const uint32_t l1 = Pl::lanes1(), l2 = Pl::lanes2();
-    uint32_t need1 = ~l1 & 31u, need2 = ~l2 & 31u;
-    uint32_t hi1 = l1 & ~31u, hi2 = l2 & ~31u;
-    for (int c = 5; c < 32; ++c) {
-      const uint32_t bit = 1u << c;
-      if ((hi1 & bit) && (hi2 & bit)) {
-        int k1 = 0, k2 = 0;
-        while (!((need1 >> k1) & 1u)) ++k1;
-        while (!((need2 >> k2) & 1u)) ++k2;
-        s.S[k1] |= bit;
-        if (k2 != k1) s.S[k2] |= bit;
-        need1 &= ~(1u << k1);
-        need2 &= ~(1u << k2);
-        hi1 &= ~bit;
-        hi2 &= ~bit;
-      }
-    }
-    for (int c = 5; c < 32; ++c) {
-      const uint32_t bit = 1u << c;
-      if (hi1 & bit) {
-        int k = 0;
-        while (!((need1 >> k) & 1u)) ++k;
-        s.S[k] |= bit;
-        need1 &= ~(1u << k);
-      }
-      if (hi2 & bit) {
-        int k = 0;
-        while (!((need2 >> k) & 1u)) ++k;
-        s.S[k] |= bit;
-        need2 &= ~(1u << k);
-      }
-    }
-    return s;
-  }
-  static constexpr uint32_t S0 = solve().S[0], S1 = solve().S[1], S2 = solve().S[2], S3 = solve().S[3],
-                            S4 = solve().S[4];
-
-  static __host__ __device__ constexpr uint32_t parity(uint32_t v) {
-    v ^= v >> 16; v ^= v >> 8; v ^= v >> 4; v ^= v >> 2; v ^= v >> 1;
-    return v & 1u;
-  }
+  // Address bit that lane bit j selects in layout 2 (lane bits past the block's P threads select
+  // the neighbouring block or row, i.e. address bit L, when P == 16).
+  static constexpr int lane_bit2(int j) { return (1 << j) < P ? ilog2_c(idx2(1 << j, 0)) : L; }
+  // Float swizzle: bits 0-1 untouched (128-bit stores keep 4 floats together); bit 2 ^= bit 5,
+  // bit 3 ^= first high lane bit of layout 2, bit 4 ^= the second one.
+  static constexpr int H1 = lane_bit2(3 - XB), H2 = lane_bit2(4 - XB);
   static __host__ __device__ constexpr uint32_t swz(uint32_t a) {
-    return a ^ ((parity(a & S0) << 0) | (parity(a & S1) << 1) | (parity(a & S2) << 2) | (parity(a & S3) << 3) |
-                (parity(a & S4) << 4));
+    return a ^ ((((a >> 5) & 1u) << 2) | (((a >> H1) & 1u) << 3) | (((a >> H2) & 1u) << 4));
   }
 
-  // For every register index, the 32 lanes of a warp hit 32 distinct banks.
-  static constexpr bool check_layout(int which) {
-    for (int r = 0; r < Pl::E; ++r) {
-      uint32_t seen = 0;
-      for (int lane = 0; lane < 32; ++lane) {
-        const int p = lane % (Pl::P < 32 ? Pl::P : 32);
-        const uint32_t blk = (Pl::P < 32) ? (uint32_t)(lane / Pl::P) : 0u;
-        const uint32_t a = (blk << Pl::L) | (uint32_t)(which == 1 ? Pl::idx1(p, r) : Pl::idx2(p, r));
-        const uint32_t bank = swz(a) & 31u;
-        if ((seen >> bank) & 1u) return false;
-        seen |= 1u << bank;
+  // Exhaustive compile-time check of bank conflicts: layout-1 128-bit stores (the 8 lanes of a
+  // phase must hit distinct 16-byte groups) and layout-2 scalar loads (32 lanes on distinct
+  // banks; a two-way conflict is unavoidable when index bit 0 is a register bit).
+  static constexpr uint32_t addr(int which, int lane, int r) {
+    const int p = lane % (P < 32 ? P : 32);
+    const uint32_t blk = (P < 32) ? (uint32_t)(lane / P) : 0u;
+    return swz((blk << L) | (uint32_t)(which == 1 ? idx1(p, r) : idx2(p, r)));
+  }
+  static constexpr bool check_store1() {
+    for (int r = 0; r < E; r += 4)
+      for (int ph = 0; ph < 4; ++ph) {
+        uint32_t seen = 0;
+        for (int l = 8 * ph; l < 8 * ph + 8; ++l) {
+          const uint32_t g = (addr(1, l, r) >> 2) & 7u;
+          if ((seen >> g) & 1u) return false;
+          seen |= 1u << g;
+        }
       }
-    }
     return true;
   }
-  static_assert(check_layout(1) && check_layout(2), "shared-memory swizzle has bank conflicts");
+  static constexpr int load2_ways() {
+    int worst = 1;
+    for (int r = 0; r < E; ++r) {
+      int cnt[32] = {0};
+      for (int l = 0; l < 32; ++l) {
+        const int b = (int)(addr(2, l, r) & 31u);
+        if (++cnt[b] > worst) worst = cnt[b];
+      }
+    }
+    return worst;
+  }
 };
 
 // ---------------------------------------------------------------- register butterflies
 
-// Butterfly stages h = 1, 2, 4, ..., < (1 << NSTAGE) over a register array (Sylvester order:
-// (a, b) at (j, j+h) becomes (a + b, a - b)).
+// Butterfly stages on register-index bits 0 .. NSTAGE-1 of v (E values stored as E/2 float2;
+// register r lives in v[r >> 1].x/.y). Sylvester order: (a, b) at (j, j+h) becomes (a+b, a-b).
 template <int E, int NSTAGE>
-__device__ __forceinline__ void fwht_regs(float (&v)[E]) {
+__device__ __forceinline__ void fwht_regs2(float2 (&v)[E / 2]) {
+  // register bit 0: the two halves of each float2
 #pragma unroll
-  for (int h = 1; h < (1 << NSTAGE); h <<= 1) {
+  for (int j = 0; j < E / 2; ++j) {
+    const float a = v[j].x, b = v[j].y;
+    v[j].x = a + b;
+    v[j].y = a - b;
+  }
+  const float2 neg1 = make_float2(-1.f, -1.f);
 #pragma unroll
-    for (int j = 0; j < E; ++j) {
+  for (int h = 1; h < (1 << (NSTAGE - 1)); h <<= 1) {  // register bits 1.. -> float2 index bits
+#pragma unroll
+    for (int j = 0; j < E / 2; ++j) {
       if ((j & h) == 0) {
-        const float a = v[j], b = v[j + h];
-        v[j] = a + b;
-        v[j + h] = a - b;
+        const float2 a = v[j], b = v[j + h];
+        v[j] = __fadd2_rn(a, b);
+        v[j + h] = __ffma2_rn(b, neg1, a);  // a - b, exactly rounded
       }
     }
-  }
-}
-
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& w, float* f) {
-  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(u[i] << 16);
-    f[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
   }
 }
 
 // ---------------------------------------------------------------- the kernel
 
 // Largest CTA a plan is launched with (bounds the register budget of the big transforms).
-constexpr int nfq_max_threads(int L) { return L >= 13 ? 256 : (L >= 11 ? 512 : 1024); }
+constexpr int nfq_max_threads(int L) { return L >= 11 ? 256 : 512; }
 
-template <int L, int EB, int R, bool HAS_GAIN>
+// QM: 0 = a8 absmax, 1 = a4 absmean, 2 = a4 absmax
+template <int L, int EB, int R, bool HAS_GAIN, int QM>
 __global__ void __launch_bounds__(nfq_max_threads(L)) norm_fht_quant_kernel(const NfqArgs a) {
   using Pl = FhtPlan<L, EB>;
-  using Sw = FhtSwizzle<Pl>;
-  constexpr int n = Pl::n, P = Pl::P, E = Pl::E, NV = Pl::NV;
-  extern __shared__ __align__(16) float smem_f[];
+  static_assert(Pl::check_store1(), "layout-1 stores have bank conflicts");
+  static_assert(Pl::load2_ways() <= (Pl::XB ? 2 : 1), "layout-2 loads have avoidable bank conflicts");
+  constexpr int n = Pl::n, P = Pl::P, E = Pl::E, NV = Pl::NV, S2 = Pl::S2, XB = Pl::XB;
+  extern __shared__ __align__(128) uint8_t smem_nfq[];
   __shared__ float red_ss[32], red_st[32];
+  __shared__ __align__(8) uint64_t land_bar;
+  __shared__ volatile int abort_flag;
+
+  const int K = a.K, nb = a.nb, rows = a.rows;
+  uint16_t* land = reinterpret_cast<uint16_t*>(smem_nfq);                   // rows*K bf16
+  float* fbuf = reinterpret_cast<float*>(smem_nfq + (size_t)rows * K * 2);  // rows*K fp32
+  uint8_t* cbuf = reinterpret_cast<uint8_t*>(fbuf);                         // codes, aliases fbuf
+  const int crow = K / 8 + 16;  // byte stride of one (k mod 8) row of the code matrix (padded)
 
   const int tid = threadIdx.x;
   const int tpr = a.slots * P;
@@ -215,183 +170,264 @@ __global__ void __launch_bounds__(nfq_max_threads(L)) norm_fht_quant_kernel(cons
   const int tr = tid - rloc * tpr;
   const int slot = tr / P;
   const int pt = tr - slot * P;
-  const int row = blockIdx.x * a.rows + rloc;
-  const bool live_row = row < a.M;
-  const int K = a.K, nb = a.nb;
+  const int lane = tid & 31, warp = tid >> 5;
 
-  float v[R][E];
-  float ss = 0.f;
+  constexpr float kQ = QM == 0 ? 127.f : (QM == 1 ? 2.6457513110645906f : 7.f);
+  constexpr int kLo = QM == 0 ? -128 : -8, kHi = QM == 0 ? 127 : 7;
+  constexpr bool kAbsmax = QM != 1;
 
-  // 1. load (layout 1) + sum of squares (+ gain), then in-register stages
-#pragma unroll
-  for (int rho = 0; rho < R; ++rho) {
-    const int blk = slot + rho * a.slots;
-    const bool live = live_row && blk < nb;
-    const uint16_t* src = a.X + (size_t)row * K + (size_t)blk * n + (pt << 3);
-#pragma unroll
-    for (int vv = 0; vv < NV; ++vv) {
-      float f[8];
-      if (live) {
-        const uint4 w = __ldcs(reinterpret_cast<const uint4*>(src + (vv << Pl::TOP)));
-        bf16x8_to_f32(w, f);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = 0.f;
-      }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        ss = fmaf(f[e], f[e], ss);
-        if constexpr (HAS_GAIN) {
-          if (live) f[e] *= __ldg(a.gain + (size_t)blk * n + (vv << Pl::TOP) + (pt << 3) + e);
-        }
-        v[rho][vv * 8 + e] = f[e];
-      }
-    }
-    fwht_regs<E, EB>(v[rho]);
-  }
-
-  // 2. regroup through shared memory. The swizzle acts on the float index inside the CTA's
-  // buffer, (rloc * nb + blk) * n + i; the block part has no bits below L, so the swizzle of
-  // the thread's part and of the (compile-time) register part combine by XOR.
-  const uint32_t rowbase = (uint32_t)rloc * (uint32_t)K;
-#pragma unroll
-  for (int rho = 0; rho < R; ++rho) {
-    const int blk = slot + rho * a.slots;
-    if (blk < nb) {
-      const uint32_t tb = rowbase + ((uint32_t)blk << L) + ((uint32_t)pt << 3);
-      const uint32_t tbs = Sw::swz(tb);
-#pragma unroll
-      for (int r = 0; r < E; ++r) {
-        const uint32_t rc = (uint32_t)Pl::idx1(0, r);
-        smem_f[tbs ^ Sw::swz(rc)] = v[rho][r];
-      }
-    }
+  if (tid == 0) {
+    abort_flag = 0;
+    mbar_init(&land_bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-#pragma unroll
-  for (int rho = 0; rho < R; ++rho) {
-    const int blk = slot + rho * a.slots;
-    if (blk < nb) {
-      const uint32_t tb = rowbase + ((uint32_t)blk << L) + (uint32_t)Pl::idx2(pt, 0);
-      const uint32_t tbs = Sw::swz(tb);
-#pragma unroll
-      for (int r = 0; r < E; ++r) {
-        const uint32_t rc = (uint32_t)Pl::idx2(0, r);
-        v[rho][r] = smem_f[tbs ^ Sw::swz(rc)];
-      }
-      fwht_regs<E, Pl::S2>(v[rho]);
-    } else {
-#pragma unroll
-      for (int r = 0; r < E; ++r) v[rho][r] = 0.f;
-    }
-  }
 
-  // 3. row statistics
-  const bool use_max = (a.quant != 1);
-  float st = 0.f;
-#pragma unroll
-  for (int rho = 0; rho < R; ++rho) {
-#pragma unroll
-    for (int r = 0; r < E; ++r) {
-      const float m = fabsf(v[rho][r]);
-      st = use_max ? fmaxf(st, m) : st + m;
-    }
+  int g = blockIdx.x;
+  if (tid == 0 && g < a.groups) {
+    const int nr = min(rows, a.M - g * rows);
+    const uint32_t bytes = (uint32_t)nr * (uint32_t)K * 2u;
+    mbar_arrive_expect_tx(&land_bar, bytes);
+    bulk_load_1d(land, a.X + (size_t)g * rows * K, bytes, &land_bar);
   }
-  const int lane = tid & 31, warp = tid >> 5;
-  if (tpr >= 32) {
+  bool pending = g < a.groups;
+  uint32_t phase = 0;
+
+  for (; g < a.groups; g += gridDim.x) {
+    const int row = g * rows + rloc;
+    const bool live_row = row < a.M;
+
+    // ---- wait for this group's rows (every thread; bounded)
+    if (!mbar_wait(&land_bar, phase, &abort_flag)) abort_flag = 1;
+    __syncthreads();
+    if (abort_flag) break;
+    phase ^= 1u;
+    pending = false;
+
+    // ---- 1. layout 1 from the landing buffer, sum of squares (+ gain)
+    float2 v[R][E / 2];
+    float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      const float t = __shfl_xor_sync(0xffffffffu, st, o);
-      st = use_max ? fmaxf(st, t) : st + t;
+    for (int rho = 0; rho < R; ++rho) {
+      const int blk = slot + rho * a.slots;
+      const bool live = live_row && blk < nb;
+      const uint16_t* src = land + (size_t)rloc * K + (size_t)blk * n + (pt << 3);
+#pragma unroll
+      for (int vv = 0; vv < NV; ++vv) {
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (live) w = *reinterpret_cast<const uint4*>(src + (vv << Pl::TOP));
+        const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float2 f = make_float2(__uint_as_float(u[i] << 16), __uint_as_float(u[i] & 0xffff0000u));
+          ss2 = __ffma2_rn(f, f, ss2);
+          if constexpr (HAS_GAIN) {
+            if (live) {
+              const float2 gg = *reinterpret_cast<const float2*>(a.gain + (size_t)blk * n + (vv << Pl::TOP) +
+                                                                 (pt << 3) + 2 * i);
+              f = __fmul2_rn(f, gg);
+            }
+          }
+          v[rho][vv * 4 + i] = f;
+        }
+      }
     }
-    if (lane == 0) {
-      red_ss[warp] = ss;
-      red_st[warp] = st;
+    __syncthreads();  // landing buffer consumed: prefetch the next group
+    const int gn = g + (int)gridDim.x;
+    if (tid == 0 && gn < a.groups) {
+      const int nr = min(rows, a.M - gn * rows);
+      const uint32_t bytes = (uint32_t)nr * (uint32_t)K * 2u;
+      mbar_arrive_expect_tx(&land_bar, bytes);
+      bulk_load_1d(land, a.X + (size_t)gn * rows * K, bytes, &land_bar);
+    }
+    pending = gn < a.groups;
+    float ss = ss2.x + ss2.y;
+
+#pragma unroll
+    for (int rho = 0; rho < R; ++rho) fwht_regs2<E, EB>(v[rho]);
+
+    // ---- 2. regroup through shared memory (index within the CTA buffer: (rloc*nb + blk)*n + i)
+    const uint32_t rowbase = (uint32_t)rloc * (uint32_t)K;
+#pragma unroll
+    for (int rho = 0; rho < R; ++rho) {
+      const int blk = slot + rho * a.slots;
+      if (blk < nb) {
+        const uint32_t tb = rowbase + ((uint32_t)blk << L) + ((uint32_t)pt << 3);
+        const uint32_t tbs = Pl::swz(tb);
+#pragma unroll
+        for (int r = 0; r < E; r += 4) {
+          const uint32_t rc = (uint32_t)Pl::idx1(0, r);
+          const float4 q4 = make_float4(v[rho][r / 2].x, v[rho][r / 2].y, v[rho][r / 2 + 1].x, v[rho][r / 2 + 1].y);
+          *reinterpret_cast<float4*>(fbuf + (tbs ^ Pl::swz(rc))) = q4;
+        }
+      }
     }
     __syncthreads();
-    const int w0 = (rloc * tpr) >> 5, nw = tpr >> 5;
-    ss = 0.f;
-    st = 0.f;
-    for (int w = 0; w < nw; ++w) {  // fixed order: identical result in every thread of the row
-      ss += red_ss[w0 + w];
-      st = use_max ? fmaxf(st, red_st[w0 + w]) : st + red_st[w0 + w];
-    }
-  } else {  // 16 threads per row, two rows per warp
 #pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) {
-      ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      const float t = __shfl_xor_sync(0xffffffffu, st, o);
-      st = use_max ? fmaxf(st, t) : st + t;
-    }
-    __syncthreads();  // every layout-2 read is done before codes overwrite shared memory
-  }
-
-  // 4. per-row multiplier and scale
-  float qmax, lo, hi;
-  if (a.quant == 0) { qmax = 127.f; lo = -128.f; hi = 127.f; }
-  else if (a.quant == 1) { qmax = 2.6457513110645906f; lo = -8.f; hi = 7.f; }
-  else { qmax = 7.f; lo = -8.f; hi = 7.f; }
-  const float r_rms = sqrtf(ss / (float)K + a.eps_norm);
-  const float rs = r_rms * sqrtf((float)n);           // y = xr * rs  (xr = orthonormal output)
-  const float sy = use_max ? st : st / (float)K;     // statistic of y
-  float mult, sx;
-  if (a.eps_q == 0.f) {
-    mult = sy > 0.f ? qmax / sy : 0.f;
-    sx = sy > 0.f ? sy / (rs * qmax) : 0.f;
-  } else {
-    const float stat = sy / rs;                        // statistic of xr
-    mult = qmax / ((stat + a.eps_q) * rs);
-    sx = stat / qmax;
-  }
-  if (live_row && tr == 0) a.s_x[row] = sx;
-
-  // 5. codes -> shared bytes (swizzled), layout-2 positions
-  uint8_t* sbytes = reinterpret_cast<uint8_t*>(smem_f);
+    for (int rho = 0; rho < R; ++rho) {
+      const int blk = slot + rho * a.slots;
+      if (blk < nb) {
+        const uint32_t tb = rowbase + ((uint32_t)blk << L) + (uint32_t)Pl::idx2(pt, 0);
+        const uint32_t tbs = Pl::swz(tb);
 #pragma unroll
-  for (int rho = 0; rho < R; ++rho) {
-    const int blk = slot + rho * a.slots;
-    if (blk < nb) {
+        for (int r = 0; r < E; r += 2) {
+          v[rho][r / 2].x = fbuf[tbs ^ Pl::swz((uint32_t)Pl::idx2(0, r))];
+          v[rho][r / 2].y = fbuf[tbs ^ Pl::swz((uint32_t)Pl::idx2(0, r + 1))];
+        }
+        fwht_regs2<E, S2>(v[rho]);
+      } else {
 #pragma unroll
-      for (int r = 0; r < E; ++r) {
-        float q = __fmul_rn(v[rho][r], mult);
-        q = fminf(fmaxf(q, lo), hi);
-        const int qi = __float2int_rn(q);
-        const uint32_t ba = rowbase + ((uint32_t)blk << L) + (uint32_t)Pl::idx2(pt, r);
-        sbytes[Pl::bswz(ba)] = (uint8_t)(qi & 0xff);
+        for (int r = 0; r < E / 2; ++r) v[rho][r] = make_float2(0.f, 0.f);
       }
     }
-  }
-  __syncthreads();
 
-  // 6. stream codes out in natural order
-  const int chunks = a.rows * K / 16;
-  const bool packed4 = (a.fmt == 0) && (a.quant != 0);
-  for (int c = tid; c < chunks; c += blockDim.x) {
-    const uint32_t off = (uint32_t)c * 16;
-    const int rl = (int)(off / (uint32_t)K);
-    const int col = (int)(off - (uint32_t)rl * K);
-    const int grow = blockIdx.x * a.rows + rl;
-    if (grow >= a.M) continue;
-    const uint2 lo8 = *reinterpret_cast<const uint2*>(sbytes + Pl::bswz(off));
-    const uint2 hi8 = *reinterpret_cast<const uint2*>(sbytes + Pl::bswz(off + 8));
-    if (!packed4) {
-      uint4 o = make_uint4(lo8.x, lo8.y, hi8.x, hi8.y);
-      *reinterpret_cast<uint4*>(a.codes + (size_t)grow * K + col) = o;
+    // ---- 3. row statistics
+    float st = 0.f;
+#pragma unroll
+    for (int rho = 0; rho < R; ++rho) {
+#pragma unroll
+      for (int r = 0; r < E / 2; ++r) {
+        if constexpr (kAbsmax) st = fmaxf(st, fmaxf(fabsf(v[rho][r].x), fabsf(v[rho][r].y)));
+        else st += fabsf(v[rho][r].x) + fabsf(v[rho][r].y);
+      }
+    }
+    if (tpr >= 32) {
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) {
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float t = __shfl_xor_sync(0xffffffffu, st, o);
+        st = kAbsmax ? fmaxf(st, t) : st + t;
+      }
+      if (lane == 0) {
+        red_ss[warp] = ss;
+        red_st[warp] = st;
+      }
+      __syncthreads();
+      const int w0 = (rloc * tpr) >> 5, nw = tpr >> 5;
+      ss = 0.f;
+      st = 0.f;
+      for (int w = 0; w < nw; ++w) {  // fixed order: the same result in every thread of the row
+        ss += red_ss[w0 + w];
+        st = kAbsmax ? fmaxf(st, red_st[w0 + w]) : st + red_st[w0 + w];
+      }
+    } else {  // 16 threads per row, two rows per warp
+#pragma unroll
+      for (int o = 8; o >= 1; o >>= 1) {
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float t = __shfl_xor_sync(0xffffffffu, st, o);
+        st = kAbsmax ? fmaxf(st, t) : st + t;
+      }
+      __syncthreads();  // every layout-2 read is done before codes overwrite the buffer
+    }
+
+    // ---- 4. per-row multiplier and scale
+    const float r_rms = sqrtf(ss / (float)K + a.eps_norm);
+    const float rs = r_rms * sqrtf((float)n);        // y = xr * rs (xr = orthonormal output)
+    const float sy = kAbsmax ? st : st / (float)K;  // statistic of y
+    float mult, sx;
+    if (a.eps_q == 0.f) {
+      mult = sy > 0.f ? kQ / sy : 0.f;
+      sx = sy > 0.f ? sy / (rs * kQ) : 0.f;
     } else {
-      // bytes b0..b15 -> nibble pairs: out byte j = (b[2j] & 15) | (b[2j+1] << 4)
-      const uint32_t w[4] = {lo8.x, lo8.y, hi8.x, hi8.y};
-      uint32_t o[2];
+      const float stat = sy / rs;                     // statistic of xr
+      mult = kQ / ((stat + a.eps_q) * rs);
+      sx = stat / kQ;
+    }
+    if (live_row && tr == 0) a.s_x[row] = sx;
+
+    // ---- 5. codes: fp32 product, clamp (absmean only: absmax products already lie in
+    // [-Q, Q]), then round to nearest even by adding 1.5 * 2^23 -- the integer lands in the low
+    // mantissa bits and, being small, its low 16 bits are the int16 code. 4 codes per word,
+    // 16 bytes per store.
+    const float2 mult2 = make_float2(mult, mult);
+    const float2 magic2 = make_float2(12582912.f, 12582912.f);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t x0 = w[2 * h], x1 = w[2 * h + 1];
-        const uint32_t e0 = (x0 & 0x0fu) | ((x0 >> 4) & 0xf0u);             // bytes 0,1
-        const uint32_t e1 = ((x0 >> 16) & 0x0fu) | ((x0 >> 20) & 0xf0u);   // bytes 2,3
-        const uint32_t e2 = (x1 & 0x0fu) | ((x1 >> 4) & 0xf0u);
-        const uint32_t e3 = ((x1 >> 16) & 0x0fu) | ((x1 >> 20) & 0xf0u);
-        o[h] = e0 | (e1 << 8) | (e2 << 16) | (e3 << 24);
+    for (int rho = 0; rho < R; ++rho) {
+      const int blk = slot + rho * a.slots;
+      if (blk < nb) {
+#pragma unroll
+        for (int x = 0; x < (1 << XB); ++x) {
+          // codes of registers r = (x << S2) | j are those of k = 8 * (c0 + j) + b
+          const int b = x | ((pt & ((1 << (3 - XB)) - 1)) << XB);
+          const int c0 = (blk << (L - 3)) + ((pt >> (3 - XB)) << (Pl::TOP - 3));
+          uint8_t* dst = cbuf + (size_t)rloc * 8 * crow + (size_t)b * crow + c0;
+#pragma unroll
+          for (int j = 0; j < (1 << S2); j += 16) {
+            uint32_t wds[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int r0 = (x << S2) + j + 4 * q;  // 4 consecutive registers = 2 float2
+              float2 t0 = __fmul2_rn(v[rho][r0 / 2], mult2);
+              float2 t1 = __fmul2_rn(v[rho][r0 / 2 + 1], mult2);
+              if constexpr (!kAbsmax) {
+                t0.x = fminf(fmaxf(t0.x, (float)kLo), (float)kHi);
+                t0.y = fminf(fmaxf(t0.y, (float)kLo), (float)kHi);
+                t1.x = fminf(fmaxf(t1.x, (float)kLo), (float)kHi);
+                t1.y = fminf(fmaxf(t1.y, (float)kLo), (float)kHi);
+              }
+              const float2 p0 = __fadd2_rn(t0, magic2);
+              const float2 p1 = __fadd2_rn(t1, magic2);
+              const uint32_t h0 = __byte_perm(__float_as_uint(p0.x), __float_as_uint(p0.y), 0x5410);
+              const uint32_t h1 = __byte_perm(__float_as_uint(p1.x), __float_as_uint(p1.y), 0x5410);
+              wds[q] = __byte_perm(h0, h1, 0x6420);
+            }
+            *reinterpret_cast<uint4*>(dst + j) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+          }
+        }
       }
-      *reinterpret_cast<uint2*>(a.codes + (size_t)grow * (K / 2) + col / 2) = make_uint2(o[0], o[1]);
+    }
+    __syncthreads();
+
+    // ---- 6. stream codes out in natural order, 32 consecutive codes per unit
+    const int upr = K / 32;  // units per row
+    const bool packed4 = (a.fmt == 0) && (QM != 0);
+    for (int u = tid; u < rows * upr; u += blockDim.x) {
+      const int rl = u / upr;
+      const int vcol = u - rl * upr;
+      const int grow = g * rows + rl;
+      if (grow >= a.M) continue;
+      const uint8_t* srcc = cbuf + (size_t)rl * 8 * crow + 4 * vcol;
+      uint32_t w[8];
+#pragma unroll
+      for (int b = 0; b < 8; ++b) w[b] = *reinterpret_cast<const uint32_t*>(srcc + (size_t)b * crow);
+      // byte j of w[b] is the code of k = 32 * vcol + 8 * j + b
+      if (!packed4) {
+        uint32_t o[8];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // k mod 8 = 4h .. 4h+3
+          const uint32_t a01l = __byte_perm(w[4 * h], w[4 * h + 1], 0x5140);
+          const uint32_t a01h = __byte_perm(w[4 * h], w[4 * h + 1], 0x7362);
+          const uint32_t a23l = __byte_perm(w[4 * h + 2], w[4 * h + 3], 0x5140);
+          const uint32_t a23h = __byte_perm(w[4 * h + 2], w[4 * h + 3], 0x7362);
+          o[0 + h] = __byte_perm(a01l, a23l, 0x5410);  // j = 0
+          o[2 + h] = __byte_perm(a01l, a23l, 0x7632);  // j = 1
+          o[4 + h] = __byte_perm(a01h, a23h, 0x5410);  // j = 2
+          o[6 + h] = __byte_perm(a01h, a23h, 0x7632);  // j = 3
+        }
+        uint4* dstg = reinterpret_cast<uint4*>(a.codes + (size_t)grow * K + 32 * vcol);
+        dstg[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        dstg[1] = make_uint4(o[4], o[5], o[6], o[7]);
+      } else {
+        // nibble pairs first: byte j of m[i] = code(8j + 2i) | code(8j + 2i + 1) << 4
+        uint32_t m[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m[i] = (w[2 * i] & 0x0f0f0f0fu) | ((w[2 * i + 1] & 0x0f0f0f0fu) << 4);
+        const uint32_t a01l = __byte_perm(m[0], m[1], 0x5140);
+        const uint32_t a01h = __byte_perm(m[0], m[1], 0x7362);
+        const uint32_t a23l = __byte_perm(m[2], m[3], 0x5140);
+        const uint32_t a23h = __byte_perm(m[2], m[3], 0x7362);
+        const uint4 o = make_uint4(__byte_perm(a01l, a23l, 0x5410), __byte_perm(a01l, a23l, 0x7632),
+                                   __byte_perm(a01h, a23h, 0x5410), __byte_perm(a01h, a23h, 0x7632));
+        *reinterpret_cast<uint4*>(a.codes + (size_t)grow * (K / 2) + 16 * vcol) = o;
+      }
+    }
+    // the next iteration's first __syncthreads orders these reads before the buffer is rewritten
+  }
+
+  // an early exit must not leave a copy in flight into shared memory
+  if (tid == 0 && pending) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(&land_bar, phase) && globaltimer_ns() - t0 < kWaitLimitNs) {
     }
   }
 }
