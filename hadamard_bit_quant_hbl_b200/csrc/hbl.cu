@@ -50,7 +50,8 @@ int device_sms(int dev) {
 }
 
 // Raise a kernel's dynamic shared memory limit when a launch needs more than was allowed so far
-// on the current device (the limit does not change occupancy; the launch's own size does).
+// on the current device (the limit does not change occupancy; the launch's own size does). The
+// default limit counts static shared memory too, so it is raised for any non-zero size.
 struct SmemLimit {
   std::mutex mu;
   int allowed[64] = {0};
@@ -58,7 +59,6 @@ struct SmemLimit {
 
 template <typename F>
 cudaError_t allow_smem(F* kernel, int bytes, SmemLimit& lim) {
-  if (bytes <= 48 * 1024) return cudaSuccess;
   int dev = 0;
   cudaGetDevice(&dev);
   dev &= 63;
