@@ -467,3 +467,66 @@ hbl_status hbl_forward(const void* X, const float* gain, const void* packed, siz
 }
 
 }  // extern "C"
+
+// =========================================================================== forward without a
+// caller-provided workspace
+//
+// Some callers cannot call cudaMalloc: host code whose device memory is owned by another
+// component's allocator (and may not allocate behind its back), or a runtime that makes all of its
+// device allocations once at start-up and none on the request path. For them hbl_forward_static
+// runs the same forward pass with its scratch (activation codes and per-token scales) in a
+// fixed-size array that is part of the library's device image. Every GPU that loads the library
+// holds this array until the process exits.
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;  // 16 MiB per device
+
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+struct StaticScratch {
+  std::mutex mu;
+  void* addr[kMaxDevices] = {nullptr};
+};
+
+StaticScratch& static_scratch() {
+  static StaticScratch s;
+  return s;
+}
+
+// Device address of g_static_scratch on the current device (looked up once per device; host
+// code only sees a host-side stand-in for the array's name, never its device address).
+hbl_status static_scratch_addr(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return HBL_EUNSUPPORTED;
+  StaticScratch& s = static_scratch();
+  std::lock_guard<std::mutex> lk(s.mu);
+  if (!s.addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    s.addr[dev] = p;
+  }
+  *out = s.addr[dev];
+  return HBL_OK;
+}
+
+}  // namespace
+
+extern "C" hbl_status hbl_forward_static(const void* X, const float* gain, const void* packed,
+                                         size_t packed_bytes, float alpha, int M, int K, int N,
+                                         int had_block, hbl_quant quant, float eps_norm, float eps_q,
+                                         void* Y, hbl_out_dtype out_dtype, hbl_stream_t stream) {
+  if (!dims_ok(M, K)) return HBL_EINVAL;
+  const size_t need = hbl_forward_workspace(M, K, quant);
+  if (need > kStaticScratchBytes) return HBL_EINVAL;  // request larger than the static scratch
+  void* ws = nullptr;
+  const hbl_status st = static_scratch_addr(&ws);
+  if (st != HBL_OK) return st;
+  // The kernels overwrite every scratch byte they later read (codes, then scales), so nothing
+  // has to be cleared between calls.
+  return hbl_forward(X, gain, packed, packed_bytes, alpha, M, K, N, had_block, quant, eps_norm, eps_q, ws,
+                     kStaticScratchBytes, Y, out_dtype, stream);
+}

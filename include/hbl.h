@@ -167,6 +167,29 @@ hbl_status hbl_forward(const void* X, const float* gain, const void* packed, siz
                        float eps_norm, float eps_q, void* workspace, size_t ws_bytes, void* Y,
                        hbl_out_dtype out_dtype, hbl_stream_t stream);
 
+/* ---------------------------------------------------------------------------------------
+ * hbl_forward without a caller-provided workspace. This entry point has no counterpart in the
+ * method's description; it exists for callers that cannot call cudaMalloc, e.g. host code whose
+ * device memory belongs to another component's allocator, or a runtime that allocates device
+ * memory only at start-up and never on the request path.
+ *
+ * Same arguments and result as hbl_forward, minus workspace/ws_bytes. The scratch (activation
+ * codes and per-token scales, hbl_forward_workspace(M, K, quant) bytes) lives in a 16 MiB array
+ * inside the library's device image (a static __device__ array): every GPU that loads the library
+ * holds those 16 MiB until the process exits, and no call allocates or frees device memory.
+ *   - Requests needing more than 16 MiB of scratch (roughly M * K > 16.7 million) return
+ *     HBL_EINVAL; use hbl_forward with your own workspace for them.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *     with that device current; make that first call before any stream capture.
+ *   - All calls on a device share the one array, and each call leaves its scratch contents
+ *     behind. Calls that may overlap on the GPU (different streams without ordering between
+ *     them) race on it: serialise them, or use hbl_forward.
+ * Asynchronous, like hbl_forward. */
+hbl_status hbl_forward_static(const void* X, const float* gain, const void* packed,
+                              size_t packed_bytes, float alpha, int M, int K, int N, int had_block,
+                              hbl_quant quant, float eps_norm, float eps_q, void* Y,
+                              hbl_out_dtype out_dtype, hbl_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
