@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "gemm_decode.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_tc2.cuh"
 #include "norm_fht_quant.cuh"
 #include "pack_weights.cuh"
 
@@ -267,8 +268,38 @@ hbl_status run_tc(const void* codes_i8, const int8_t* w_i8, const TcArgs& a0, cu
   return HBL_OK;
 }
 
+hbl_status run_tc2(const void* codes_i8, const int8_t* w_i8, const TcArgs& a0, cudaStream_t s) {
+  CUtensorMap mA, mB;
+  if (!make_map_i8(&mA, codes_i8, a0.K, a0.M, 128)) return HBL_ECUDA;
+  if (!make_map_i8(&mB, w_i8, a0.K, a0.N, 128)) return HBL_ECUDA;
+  Tc2Args a;
+  a.s_x = a0.s_x;
+  a.alpha = a0.alpha;
+  a.M = a0.M;
+  a.N = a0.N;
+  a.K = a0.K;
+  a.Y = a0.Y;
+  a.out_bf16 = a0.out_bf16;
+  a.acc_debug = a0.acc_debug;
+  a.tiles_m = (a.M + kT2BM - 1) / kT2BM;
+  a.tiles_n = (a.N + kT2BN - 1) / kT2BN;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int ntiles = a.tiles_m * a.tiles_n;
+  const int pairs = device_sms(dev) / 2;
+  const int grid = 2 * (ntiles < pairs ? ntiles : pairs);
+  static SmemLimit lim;
+  const cudaError_t e = allow_smem(gemm_tc2_kernel, kT2Smem, lim);
+  if (e != cudaSuccess) return cuda_fail(e);
+  gemm_tc2_kernel<<<grid, kT2Threads, kT2Smem, s>>>(mA, mB, a);
+  HBL_CHECK_LAUNCH();
+  return HBL_OK;
+}
+
 // Token counts up to this bound run on CUDA cores over the 2-bit weights.
 constexpr int kDecodeMaxM = 8;
+// From this token count on, the product runs on SM pairs (256 x 256 tiles).
+constexpr int kPairMinM = 256;
 
 hbl_status run_gemm(const void* codes, int fmt, int abits, const float* s_x, const void* packed, float alpha,
                     int M, int N, int K, void* Y, int out_dtype, int32_t* acc_debug, cudaStream_t s) {
@@ -301,7 +332,8 @@ hbl_status run_gemm(const void* codes, int fmt, int abits, const float* s_x, con
   t.Y = Y;
   t.out_bf16 = out_dtype == HBL_OUT_BF16;
   t.acc_debug = acc_debug;
-  return run_tc(codes, reinterpret_cast<const int8_t*>(blob + bl.off1), t, s);
+  const int8_t* w8 = reinterpret_cast<const int8_t*>(blob + bl.off1);
+  return M >= kPairMinM ? run_tc2(codes, w8, t, s) : run_tc(codes, w8, t, s);
 }
 
 size_t forward_codes_bytes(int M, int K) { return round_up((size_t)M * K, 256); }

@@ -114,6 +114,25 @@ struct FhtPlan {
   }
 };
 
+// Swizzled float index swz(tb) ^ swz(rc) for a runtime thread part tb and compile-time register
+// parts rc. Only bits 2..4 of the two swizzled parts overlap (the swizzle mixes nothing else), so
+// the thread keeps 8 bases, one per value of those bits, and each access is base + constant:
+// the constant folds into the load/store offset instead of costing an XOR per access.
+template <class Pl>
+struct SwzBases {
+  uint32_t b[8];
+  __device__ __forceinline__ explicit SwzBases(uint32_t tb) {
+    const uint32_t t = Pl::swz(tb);
+#pragma unroll
+    for (uint32_t c = 0; c < 8; ++c) b[c] = (t & ~0x1cu) | ((((t >> 2) & 7u) ^ c) << 2);
+  }
+  // index of register part rc (a compile-time constant after unrolling)
+  __device__ __forceinline__ uint32_t at(uint32_t rc) const {
+    const uint32_t r = Pl::swz(rc);
+    return b[(r >> 2) & 7u] + (r & ~0x1cu);
+  }
+};
+
 // ---------------------------------------------------------------- register butterflies
 
 // Butterfly stages on register-index bits 0 .. NSTAGE-1 of v (E values stored as E/2 float2;
@@ -206,7 +225,7 @@ __global__ void __launch_bounds__(nfq_max_threads(L)) norm_fht_quant_kernel(cons
 
     // ---- 1. layout 1 from the landing buffer, sum of squares (+ gain)
     float2 v[R][E / 2];
-    float2 ss2 = make_float2(0.f, 0.f);
+    float2 ss2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
     for (int rho = 0; rho < R; ++rho) {
       const int blk = slot + rho * a.slots;
@@ -220,7 +239,7 @@ __global__ void __launch_bounds__(nfq_max_threads(L)) norm_fht_quant_kernel(cons
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           float2 f = make_float2(__uint_as_float(u[i] << 16), __uint_as_float(u[i] & 0xffff0000u));
-          ss2 = __ffma2_rn(f, f, ss2);
+          ss2[i] = __ffma2_rn(f, f, ss2[i]);  // independent chains
           if constexpr (HAS_GAIN) {
             if (live) {
               const float2 gg = *reinterpret_cast<const float2*>(a.gain + (size_t)blk * n + (vv << Pl::TOP) +
@@ -241,7 +260,7 @@ __global__ void __launch_bounds__(nfq_max_threads(L)) norm_fht_quant_kernel(cons
       bulk_load_1d(land, a.X + (size_t)gn * rows * K, bytes, &land_bar);
     }
     pending = gn < a.groups;
-    float ss = ss2.x + ss2.y;
+    float ss = ((ss2[0].x + ss2[0].y) + (ss2[1].x + ss2[1].y)) + ((ss2[2].x + ss2[2].y) + (ss2[3].x + ss2[3].y));
 
 #pragma unroll
     for (int rho = 0; rho < R; ++rho) fwht_regs2<E, EB>(v[rho]);
@@ -252,13 +271,11 @@ __global__ void __launch_bounds__(nfq_max_threads(L)) norm_fht_quant_kernel(cons
     for (int rho = 0; rho < R; ++rho) {
       const int blk = slot + rho * a.slots;
       if (blk < nb) {
-        const uint32_t tb = rowbase + ((uint32_t)blk << L) + ((uint32_t)pt << 3);
-        const uint32_t tbs = Pl::swz(tb);
+        const SwzBases<Pl> sb(rowbase + ((uint32_t)blk << L) + ((uint32_t)pt << 3));
 #pragma unroll
         for (int r = 0; r < E; r += 4) {
-          const uint32_t rc = (uint32_t)Pl::idx1(0, r);
           const float4 q4 = make_float4(v[rho][r / 2].x, v[rho][r / 2].y, v[rho][r / 2 + 1].x, v[rho][r / 2 + 1].y);
-          *reinterpret_cast<float4*>(fbuf + (tbs ^ Pl::swz(rc))) = q4;
+          *reinterpret_cast<float4*>(fbuf + sb.at((uint32_t)Pl::idx1(0, r))) = q4;
         }
       }
     }
@@ -267,12 +284,11 @@ __global__ void __launch_bounds__(nfq_max_threads(L)) norm_fht_quant_kernel(cons
     for (int rho = 0; rho < R; ++rho) {
       const int blk = slot + rho * a.slots;
       if (blk < nb) {
-        const uint32_t tb = rowbase + ((uint32_t)blk << L) + (uint32_t)Pl::idx2(pt, 0);
-        const uint32_t tbs = Pl::swz(tb);
+        const SwzBases<Pl> sb(rowbase + ((uint32_t)blk << L) + (uint32_t)Pl::idx2(pt, 0));
 #pragma unroll
         for (int r = 0; r < E; r += 2) {
-          v[rho][r / 2].x = fbuf[tbs ^ Pl::swz((uint32_t)Pl::idx2(0, r))];
-          v[rho][r / 2].y = fbuf[tbs ^ Pl::swz((uint32_t)Pl::idx2(0, r + 1))];
+          v[rho][r / 2].x = fbuf[sb.at((uint32_t)Pl::idx2(0, r))];
+          v[rho][r / 2].y = fbuf[sb.at((uint32_t)Pl::idx2(0, r + 1))];
         }
         fwht_regs2<E, S2>(v[rho]);
       } else {
@@ -282,14 +298,21 @@ __global__ void __launch_bounds__(nfq_max_threads(L)) norm_fht_quant_kernel(cons
     }
 
     // ---- 3. row statistics
-    float st = 0.f;
+    float sta[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent chains
 #pragma unroll
     for (int rho = 0; rho < R; ++rho) {
 #pragma unroll
       for (int r = 0; r < E / 2; ++r) {
-        if constexpr (kAbsmax) st = fmaxf(st, fmaxf(fabsf(v[rho][r].x), fabsf(v[rho][r].y)));
-        else st += fabsf(v[rho][r].x) + fabsf(v[rho][r].y);
+        float& acc = sta[(rho * (E / 2) + r) & 7];
+        if constexpr (kAbsmax) acc = fmaxf(acc, fmaxf(fabsf(v[rho][r].x), fabsf(v[rho][r].y)));
+        else acc += fabsf(v[rho][r].x) + fabsf(v[rho][r].y);
       }
+    }
+    float st;
+    if constexpr (kAbsmax) {
+      st = fmaxf(fmaxf(fmaxf(sta[0], sta[1]), fmaxf(sta[2], sta[3])), fmaxf(fmaxf(sta[4], sta[5]), fmaxf(sta[6], sta[7])));
+    } else {
+      st = ((sta[0] + sta[1]) + (sta[2] + sta[3])) + ((sta[4] + sta[5]) + (sta[6] + sta[7]));
     }
     if (tpr >= 32) {
 #pragma unroll
