@@ -404,9 +404,13 @@ __global__ void __launch_bounds__(nfq_max_threads(L)) norm_fht_quant_kernel(cons
     // ---- 6. stream codes out in natural order, 32 consecutive codes per unit
     const int upr = K / 32;  // units per row
     const bool packed4 = (a.fmt == 0) && (QM != 0);
-    for (int u = tid; u < rows * upr; u += blockDim.x) {
-      const int rl = u / upr;
-      const int vcol = u - rl * upr;
+    // thread tid handles units tid, tid + blockDim, ... of the CTA's rows * upr units; walk them
+    // row by row without dividing
+    int rl = 0, vcol = tid;
+    while (vcol >= upr && rl < rows) { vcol -= upr; ++rl; }
+    for (; rl < rows; vcol += blockDim.x) {
+      while (vcol >= upr) { vcol -= upr; ++rl; }
+      if (rl >= rows) break;
       const int grow = g * rows + rl;
       if (grow >= a.M) continue;
       const uint8_t* srcc = cbuf + (size_t)rl * 8 * crow + 4 * vcol;
