@@ -34,11 +34,22 @@ METRIC = "H-BitLinear tokens/s and effective TOPS at 7B-like shapes; % of HBM/in
 UNIT = "tokens/s"
 M_TOKENS = 8192
 LAYERS = ("wo_7b_a4", "wdown_7b_a4")
+SWEEP_TOKENS = (1, 16, 64, 512)
 WORKLOAD = ("7B-like H-BitLinear layer pair: Wo 4096->4096 + Wdown 16384->4096, a4 absmean, "
             "8192 tokens, bf16 in / bf16 out")
 # DRAM bytes per launch of the dominant kernel from an ncu capture, with the hash of the kernel
 # source it was taken on (reported as null once the source has changed).
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # profiles/gemm_tc2_wdown_7b_m8192.md: dram__bytes_read.sum + dram__bytes_write.sum
+    "gemm_tc2[wdown_7b_a4]": {"bytes": 607.685376e6 + 73.879552e6, "src": "gemm_tc2.cuh", "sha": "179b5ae7b9be7658"},
+}
+
+
+def product_kernel(M):
+    """Name and source file of the product kernel hbl_ternary_gemm runs for M tokens."""
+    if M <= 8:
+        return "gemm_decode", "gemm_decode.cuh"
+    return ("gemm_tc2", "gemm_tc2.cuh") if M >= 256 else ("gemm_tc", "gemm_tc.cuh")
 
 
 def peaks():
@@ -285,6 +296,9 @@ def run_ours(args, world, rank, local):
     h2d = sum(L["X"].numel() * 2 for L in layers)
     d2h = sum(L["Y"].numel() * 2 for L in layers)
 
+    # ---- token-count sweep of the same layer pair (CUDA-graph replay, L2 flushed before each step)
+    sweep = [] if args.no_sweep else run_sweep(layers, dev, args)
+
     st = hbl.hbl_device_status()
     if st != hbl.HBL_OK:
         raise RuntimeError(hbl.hbl_status_string(st))
@@ -301,13 +315,13 @@ def run_ours(args, world, rank, local):
         kern.append({"kernel": f"norm_fht_quant[{sp.name}]", "ms": per[2 * i], "bound": "hbm",
                      "achieved": nfq_bytes / (per[2 * i] / 1e3) / 1e9, "unit": "GB/s",
                      "frac": nfq_bytes / (per[2 * i] / 1e3) / 1e9 / hbm})
-        kern.append({"kernel": f"gemm_tc[{sp.name}]", "ms": per[2 * i + 1], "bound": "tensor",
+        kern.append({"kernel": f"{product_kernel(sp.M)[0]}[{sp.name}]", "ms": per[2 * i + 1], "bound": "tensor",
                      "achieved": gemm_ops / (per[2 * i + 1] / 1e3) / 1e12, "unit": "TOP/s",
                      "frac": gemm_ops / (per[2 * i + 1] / 1e3) / 1e12 / int8_peak_tops})
     dom = max(kern, key=lambda k: k["ms"])
     traffic = None
     rec = NCU_TRAFFIC.get(dom["kernel"])
-    if rec and rec.get("src") == src_hash("gemm_tc.cuh" if "gemm" in dom["kernel"] else "norm_fht_quant.cuh"):
+    if rec and src_hash(rec["src"]) == rec["sha"]:  # null once the kernel source has changed
         traffic = rec["bytes"]
     eff_tops = sum(2.0 * L["spec"].M * L["spec"].N * L["spec"].K for L in layers) / (ms_step / 1e3) / 1e12
 
@@ -339,10 +353,67 @@ def run_ours(args, world, rank, local):
         "e2e": ({"value": tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                  "d2h_bytes_per_step": d2h} if e2e_steps else None),
         "gpu_launches": 4 * args.steps,
+        "sweep": sweep,
         "clocks": clk.summary(),
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
+
+
+def run_sweep(layers, dev, args):
+    """Per token count M: one step = hbl_forward of Wo then Wdown on the first M rows, captured
+    in a CUDA graph; before every timed replay a 256 MB buffer is written so that weights and
+    activations come from HBM, not L2. Reports tokens/s, effective TOPS and the bandwidth on the
+    2-bit (M <= 8) or int8 weight bytes the product reads."""
+    import torch
+
+    import hadamard_bit_quant_hbl_b200 as hbl
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    out = []
+    for M in SWEEP_TOKENS:
+        bufs = []
+        for L in layers:
+            sp = L["spec"]
+            Y = torch.empty((M, sp.N), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(hbl.hbl_forward_workspace(M, sp.K, hbl.HBL_Q_A4_ABSMEAN), dtype=torch.uint8, device=dev)
+            bufs.append((L, L["X"][:M], Y, ws))
+
+        def step(s):
+            for L, X, Y, ws in bufs:
+                hbl.hbl_forward(X, L["packed"], L["alpha"], L["spec"].N, None, L["spec"].had_block,
+                                hbl.HBL_Q_A4_ABSMEAN, workspace=ws, Y=Y, out_dtype=hbl.HBL_OUT_BF16, stream=s)
+
+        cap = torch.cuda.Stream(dev)
+        with torch.cuda.stream(cap):
+            step(cap.cuda_stream)  # warm-up outside capture (one-time host setup)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            step(cap.cuda_stream)
+        torch.cuda.synchronize()
+        reps = max(20, min(args.sweep_steps, 200))
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        tot = 0.0
+        cur = torch.cuda.current_stream(dev)
+        for _ in range(reps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(cur)
+            g.replay()
+            e1.record(cur)
+            e1.synchronize()
+            tot += e0.elapsed_time(e1)
+        ms = tot / reps
+        wbytes = sum((L["spec"].K * L["spec"].N) // (4 if M <= 8 else 1) for L in layers)
+        ops = sum(2.0 * M * L["spec"].N * L["spec"].K for L in layers)
+        out.append({"M": M, "ms_per_step": ms, "tokens_per_s": M / (ms / 1e3), "effective_tops": ops / (ms / 1e3) / 1e12,
+                    "weight_bytes": wbytes, "weight_GBps": wbytes / (ms / 1e3) / 1e9,
+                    "product": "cuda-core 2-bit" if M <= 8 else ("tcgen05 pair" if M >= 256 else "tcgen05")})
+        del g
+    return out
 
 
 def main():
@@ -355,6 +426,8 @@ def main():
     ap.add_argument("--ref-step-rows", type=int, default=1, help="token rows per layer in one reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the token-count sweep")
+    ap.add_argument("--sweep-steps", type=int, default=100)
     args = ap.parse_args()
     world, rank, local = dist_setup(args.gpus) if args.impl == "ours" else (
         int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
