@@ -26,7 +26,7 @@ struct DecodeArgs {
   int m0;                // first token row handled by this launch (rows m0 .. m0+MT-1)
   int packed4;           // 1 = packed int4 rows
   const float* s_x;
-  const uint32_t* w2;    // section 0: [N][K/16] words
+  const uint32_t* w2;    // section 0: tile-major 2-bit words (see the packer)
   float alpha;
   int M, N, K;
   void* Y;
@@ -104,7 +104,9 @@ __global__ void __launch_bounds__(512) gemm_decode_kernel(const DecodeArgs a) {
 #pragma unroll
     for (int c = 0; c < COLS; ++c) {
       const int n = n0 + c;
-      wv[c] = n < a.N ? __ldcs(reinterpret_cast<const uint4*>(a.w2 + (size_t)n * (a.K / 16)) + t)
+      // words 4t .. 4t+3 of row n: k-block t/2, half t%2 of the row's 8 words in that block
+      const size_t wi = ((size_t)(n >> 7) * (a.K >> 7) + (t >> 1)) * 1024 + (size_t)(n & 127) * 8 + (t & 1) * 4;
+      wv[c] = n < a.N ? __ldcs(reinterpret_cast<const uint4*>(a.w2 + wi))
                       : make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u);  // t = 0
     }
 #pragma unroll

@@ -1,0 +1,304 @@
+// Ternary x low-bit product for small token counts (M <= 256) on the tensor cores.
+//
+//   Y[m, n] = s_x[m] * alpha * sum_k q[m, k] * t[k, n]
+//
+// The layer's product (BitNet v2 walkthrough article, section "H-BitLinear模塊"), exact in int32.
+// With few tokens the product is bound by the weight bytes, so the weights are read in their
+// 2-bit form (4x fewer bytes than int8) and widened to int8 in shared memory, and the roles are
+// swapped: 128 output features form the MMA's M side and the (padded) tokens its N side:
+//
+//   D[n, m] = sum_k t[k, n] q[m, k],   tcgen05.mma kind::i8, M = 128, N = Mt (16..256), K = 32.
+//
+// A cluster of S CTAs shares one 128-feature tile and splits K: CTA r owns a contiguous run of
+// 128-wide k-blocks. Its partial sums end in its own shared memory and are reduced across the
+// cluster through distributed shared memory, so no global workspace is needed.
+//
+//   warp 0     TMA producer: per k-block the 2-bit weight tile (4 KB contiguous in the blob's
+//              tile-major section, one bulk copy) and the activation tile (Mt rows x 128 bytes,
+//              128-byte swizzle) into an NL-stage ring.
+//   warp 1     TMEM allocation; one thread issues 4 MMAs per k-block and commits to the ring's
+//              "empty" barriers.
+//   warps 2-5  widen each 2-bit row (8 words = 128 codes c = t+1) to 128 int8 t in the
+//              128-byte-swizzled K-major layout the MMA reads (NW-stage ring), then the epilogue:
+//              tcgen05.ld of the partial sums, reduction across the cluster, dequant, store.
+// Every mbarrier wait is bounded (1 s).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "gemm_tc2.cuh"
+
+namespace hbl {
+
+constexpr int kSwNT = 128;        // output features per tile (MMA M)
+constexpr int kSwBK = 128;        // k per block
+constexpr int kSwRaw = 128 * 32;  // bytes of one 2-bit weight tile (4 KB, contiguous in the blob)
+constexpr int kSwWide = 128 * kSwBK;
+constexpr int kSwGR = 4;          // k-blocks per 2-bit copy (16 KB: few, large bulk copies)
+constexpr int kSwNR = 4;          // 2-bit copy stages (released as soon as they are widened)
+constexpr int kSwMaxNA = 8;       // activation copy stages (released by the MMA)
+constexpr int kSwMaxNW = 4;       // widened tile stages (released by the MMA)
+constexpr int kSwThreads = 224;   // 7 warps
+constexpr int kSwSmem = 200 * 1024 + 1024;
+
+struct SwapArgs {
+  const uint32_t* w2;  // 2-bit weight section, tile-major (4 KB per 128 x 128 tile)
+  const float* s_x;
+  float alpha;
+  int M, N, K;
+  int Mt;           // tokens padded to a multiple of 16 (MMA N)
+  int NA, NW;       // activation / widened ring stages
+  int GA;           // k-blocks per activation copy (about 16 KB per copy)
+  int S;            // CTAs per cluster (k split)
+  int tmem_cols;
+  void* Y;
+  int out_bf16;
+  int32_t* acc_debug;
+};
+
+__device__ __forceinline__ uint32_t idesc_i8_mn(int M, int N) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// 32 lanes x 16 consecutive 32-bit columns, waited in the same statement.
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t cluster_addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kSwThreads, 1)
+gemm_swap_kernel(const __grid_constant__ CUtensorMap mapA, const SwapArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw3[];
+  __shared__ __align__(8) uint64_t raw_full[kSwNR], raw_empty[kSwNR];
+  __shared__ __align__(8) uint64_t act_full[kSwMaxNA], act_empty[kSwMaxNA];
+  __shared__ __align__(8) uint64_t wide_full[kSwMaxNW], wide_empty[kSwMaxNW], acc_full, drain_bar;
+  __shared__ uint32_t tmem_base_slot;
+  __shared__ volatile int abort_flag;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw3) + 1023) & ~uintptr_t(1023));
+  const int NA = a.NA, NW = a.NW, Mt = a.Mt, GA = a.GA;
+  const int act_bytes = Mt * kSwBK;                 // one k-block of activations, multiple of 2048
+  const int act_stage = GA * act_bytes;             // one copy: GA k-blocks, [GA][Mt][128] swizzled
+  uint8_t* act = smem;                              // NA x act_stage
+  uint8_t* wide = act + NA * act_stage;             // NW x 16 KB (128-byte swizzle)
+  uint8_t* raw = wide + NW * kSwWide;               // NR x (GR x 4 KB)
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int S = a.S;
+  const int tile = blockIdx.x / S;
+  const int n0 = tile * kSwNT;
+  const int KB = a.K / kSwBK;
+  const int kb0 = (int)(((long)KB * rank) / S), kb1 = (int)(((long)KB * (rank + 1)) / S);
+  const int nkb = kb1 - kb0;
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < kSwNR; ++s) {
+      mbar_init(&raw_full[s], 1);
+      mbar_init(&raw_empty[s], 4);  // one lane of each widening warp
+    }
+    for (int s = 0; s < NA; ++s) {
+      mbar_init(&act_full[s], 1);
+      mbar_init(&act_empty[s], 1);
+    }
+    for (int s = 0; s < NW; ++s) {
+      mbar_init(&wide_full[s], 4);
+      mbar_init(&wide_empty[s], 1);
+    }
+    mbar_init(&acc_full, 1);
+    mbar_init(&drain_bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    tma_prefetch_desc(&mapA);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(&tmem_base_slot)), "r"(a.tmem_cols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_slot;
+
+  if (warp == 0) {
+    // ---------------- producer of the 2-bit weight tiles (runs up to kSwNR ahead)
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      for (int i = 0; i < nkb; i += kSwGR) {
+        if (!mbar_wait(&raw_empty[s], ph ^ 1u, &abort_flag)) break;
+        const uint32_t bytes = (uint32_t)min(kSwGR, nkb - i) * kSwRaw;  // tiles of one feature tile are consecutive
+        mbar_arrive_expect_tx(&raw_full[s], bytes);
+        bulk_load_1d(raw + s * (kSwGR * kSwRaw), a.w2 + ((size_t)tile * KB + kb0 + i) * 1024, bytes, &raw_full[s]);
+        if (++s == kSwNR) { s = 0; ph ^= 1u; }
+      }
+    }
+  } else if (warp == 6) {
+    // ---------------- producer of the activation tiles (runs up to NA ahead)
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      for (int i = 0; i < nkb; i += GA) {
+        if (!mbar_wait(&act_empty[s], ph ^ 1u, &abort_flag)) break;
+        mbar_arrive_expect_tx(&act_full[s], (uint32_t)act_stage);  // the box is always complete
+        tma_load_3d(act + s * act_stage, &mapA, &act_full[s], 0, 0, kb0 + i);
+        if (++s == NA) { s = 0; ph ^= 1u; }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_i8_mn(kSwNT, Mt);
+      int sa = 0, w = 0;
+      uint32_t pha = 0, phw = 0;
+      bool ok = true, any = false;
+      for (int i = 0; i < nkb; ++i) {
+        const int ja = i % GA;  // k-block within the activation copy
+        if (!mbar_wait(&wide_full[w], phw, &abort_flag)) { ok = false; break; }
+        if (ja == 0 && !mbar_wait(&act_full[sa], pha, &abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t w_addr = smem_u32(wide + w * kSwWide);
+        const uint32_t a_addr = smem_u32(act + sa * act_stage + ja * act_bytes);
+#pragma unroll
+        for (int kk = 0; kk < kSwBK / 32; ++kk)
+          mma_i8(tmem_base, smem_desc_sw128(w_addr + kk * 32), smem_desc_sw128(a_addr + kk * 32), idesc,
+                 (i | kk) != 0 ? 1u : 0u);
+        any = true;
+        mma_commit(&wide_empty[w]);
+        if (ja == GA - 1 || i == nkb - 1) {
+          mma_commit(&act_empty[sa]);
+          if (++sa == NA) { sa = 0; pha ^= 1u; }
+        }
+        if (++w == NW) { w = 0; phw ^= 1u; }
+      }
+      if (ok && any) mma_commit(&acc_full);
+      if (!ok && any) {
+        mma_commit(&drain_bar);
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&drain_bar, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else {
+    // ---------------- widen (warps 2-5, thread = weight row of the tile). A 2-bit tile is released
+    // as soon as it is in registers; the widened tiles of a batch share one proxy fence.
+    const int row = threadIdx.x - 64;  // 0..127
+    const int batch = NW / 2;
+    int s = 0, w = 0;
+    uint32_t ph = 0, phw = 0;
+    bool ok = true;
+    for (int i0 = 0; i0 < nkb && ok; i0 += batch) {
+      const int nb = min(batch, nkb - i0);
+      int w1 = w;
+      uint32_t phw1 = phw;
+      for (int j = 0; j < nb; ++j) {
+        // every lane waits (the TMA-written tile must be visible to each reader); the outcome
+        // is made uniform so that the warp stays converged
+        const int i = i0 + j, jr = i % kSwGR;  // k-block within the 2-bit copy
+        bool r = jr != 0 || mbar_wait(&raw_full[s], ph, &abort_flag);
+        if (r) r = mbar_wait(&wide_empty[w1], phw1 ^ 1u, &abort_flag);
+        if (!__all_sync(0xffffffffu, r)) { ok = false; break; }
+        const uint8_t* rp = raw + s * (kSwGR * kSwRaw) + jr * kSwRaw + row * 32;
+        const uint4 lo = *reinterpret_cast<const uint4*>(rp);
+        const uint4 hi = *reinterpret_cast<const uint4*>(rp + 16);
+        if (jr == kSwGR - 1 || i == nkb - 1) {  // the copy is consumed: hand it back
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&raw_empty[s]);
+          if (++s == kSwNR) { s = 0; ph ^= 1u; }
+        }
+        const uint32_t wd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+        uint8_t* dst = wide + w1 * kSwWide + row * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {  // word c = 16 codes k = 16c + 4s' + b, c' = t + 1 in {0,1,2}
+          uint32_t o[4];
+#pragma unroll
+          for (int sp = 0; sp < 4; ++sp) {
+            const uint32_t u = (wd[c] >> (2 * sp)) & 0x03030303u;  // c' per byte
+            o[sp] = (u + 0x7f7f7f7fu) ^ 0x80808080u;             // int8 t = c' - 1, no carries
+          }
+          *reinterpret_cast<uint4*>(dst + ((c ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        if (++w1 == NW) { w1 = 0; phw1 ^= 1u; }
+      }
+      if (!ok) break;
+      fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+      __syncwarp();
+      for (int j = 0; j < nb; ++j) {
+        if (lane == 0) mbar_arrive(&wide_full[w]);
+        if (++w == NW) { w = 0; phw ^= 1u; }
+      }
+    }
+
+    // ---------------- epilogue part 1: partial sums -> own shared memory as [Mt][128] int32
+    bool r = ok && mbar_wait(&acc_full, 0, &abort_flag);
+    r = __all_sync(0xffffffffu, r);
+    int32_t* part = reinterpret_cast<int32_t*>(smem);  // the rings are idle now
+    if (r && nkb > 0) {
+      tc_fence_after();
+      const int q = warp & 3;  // TMEM lane quarter
+      const int f = q * 32 + lane;
+      for (int c0 = 0; c0 < Mt; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) part[(c0 + j) * kSwNT + f] = (int32_t)v[j];
+      }
+    } else {
+      for (int m = 0; m < Mt; ++m) part[m * kSwNT + (warp & 3) * 32 + lane] = 0;
+    }
+  }
+
+  // ---------------- epilogue part 2: reduce the cluster's partial sums, dequant, store
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp >= 2 && warp <= 5) {
+    const uint32_t part0 = smem_u32(smem);
+    const int t = threadIdx.x - 64;
+    for (int e = (int)rank * 128 + t; e < Mt * kSwNT; e += S * 128) {
+      const int m = e / kSwNT, f = e - m * kSwNT;
+      const int n = n0 + f;
+      if (m >= a.M || n >= a.N) continue;
+      uint32_t pv[8];
+#pragma unroll
+      for (int p = 0; p < 8; ++p)  // all remote loads in flight before the sum
+        pv[p] = p < S ? ld_shared_cluster_u32(mapa_shared(part0 + (uint32_t)e * 4u, (uint32_t)p)) : 0u;
+      int32_t acc = 0;
+#pragma unroll
+      for (int p = 0; p < 8; ++p) acc += (int32_t)pv[p];  // fixed order
+      const float y = (float)acc * (a.s_x[m] * a.alpha);
+      if (a.out_bf16) reinterpret_cast<__nv_bfloat16*>(a.Y)[(size_t)m * a.N + n] = __float2bfloat16_rn(y);
+      else reinterpret_cast<float*>(a.Y)[(size_t)m * a.N + n] = y;
+      if (a.acc_debug) a.acc_debug[(size_t)m * a.N + n] = acc;
+    }
+  }
+  __syncwarp();
+  cluster_sync_all();  // no CTA leaves while a peer may still read its shared memory
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(a.tmem_cols)
+                 : "memory");
+  }
+}
+
+}  // namespace hbl

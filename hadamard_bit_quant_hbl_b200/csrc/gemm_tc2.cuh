@@ -148,6 +148,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
                  ::"r"(smem_u32(&tmem_base_slot)) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
+  __syncwarp();
   tc_fence_before();
   cluster_sync_all();  // barriers initialised and TMEM allocated in both CTAs
   tc_fence_after();
@@ -285,6 +286,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
   }
 
   // both CTAs are done with TMEM and with each other's barriers and shared memory
+  __syncwarp();
   tc_fence_before();
   cluster_sync_all();
   if (warp == 1) {

@@ -13,6 +13,7 @@
 #include "gemm_decode.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_tc2.cuh"
+#include "gemm_swap.cuh"
 #include "norm_fht_quant.cuh"
 #include "pack_weights.cuh"
 
@@ -79,7 +80,7 @@ struct BlobLayout {
 BlobLayout blob_layout(int K, int N) {
   BlobLayout b;
   b.off0 = 0;
-  b.off1 = round_up((size_t)N * K / 4, 256);
+  b.off1 = round_up((size_t)((N + 127) / 128 * 128) * K / 4, 256);  // section 0 padded to whole tiles
   b.off2 = b.off1 + round_up((size_t)N * K, 256);
   b.total = b.off2 + round_up((size_t)N * 4, 256);
   return b;
@@ -296,7 +297,78 @@ hbl_status run_tc2(const void* codes_i8, const int8_t* w_i8, const TcArgs& a0, c
   return HBL_OK;
 }
 
-// Token counts up to this bound run on CUDA cores over the 2-bit weights.
+// 3-D view of int8 codes [rows][K] as (128 bytes, rows, K/128 blocks) with a (128, box_rows, gb) box
+// and 128-byte swizzle: one copy brings gb consecutive k-blocks, laid out as [gb][box_rows][128].
+bool make_map_i8_blocks(CUtensorMap* map, const void* base, int K, int rows, int box_rows, int gb) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {128u, (cuuint64_t)rows, (cuuint64_t)(K / 128)};
+  const cuuint64_t strides[2] = {(cuuint64_t)K, 128u};
+  const cuuint32_t box[3] = {128u, (cuuint32_t)box_rows, (cuuint32_t)gb};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Products for up to this many tokens run on the swapped tensor-core kernel over 2-bit weights.
+constexpr int kSwapMaxM = 256;
+
+hbl_status run_swap(const void* codes_i8, const void* w2, const TcArgs& t, cudaStream_t s) {
+  SwapArgs a;
+  a.s_x = t.s_x;
+  a.alpha = t.alpha;
+  a.M = t.M;
+  a.N = t.N;
+  a.K = t.K;
+  a.Mt = (t.M + 15) / 16 * 16;
+  // activation copies of about 16 KB; shared memory: 4 x 16 KB of 2-bit tiles, NW x 16 KB
+  // widened tiles, the rest activation copies
+  a.GA = a.Mt >= 128 ? 1 : 128 / a.Mt;
+  a.NW = a.Mt <= 128 ? kSwMaxNW : 3;
+  a.NA = (200 * 1024 - kSwNR * kSwGR * kSwRaw - a.NW * kSwWide) / (a.GA * a.Mt * kSwBK);
+  if (a.NA > kSwMaxNA) a.NA = kSwMaxNA;
+  int cols = 32;
+  while (cols < a.Mt) cols *= 2;
+  a.tmem_cols = cols;
+  a.Y = t.Y;
+  a.out_bf16 = t.out_bf16;
+  a.acc_debug = t.acc_debug;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int ntiles = (a.N + kSwNT - 1) / kSwNT;
+  const int KB = a.K / kSwBK;
+  int S = device_sms(dev) / ntiles;  // split K so that the grid fills the device
+  if (S > 8) S = 8;
+  if (S > KB) S = KB;
+  if (S < 1) S = 1;
+  a.S = S;
+  a.w2 = static_cast<const uint32_t*>(w2);
+  CUtensorMap mA;
+  if (!make_map_i8_blocks(&mA, codes_i8, a.K, a.M, a.Mt, a.GA)) return HBL_ECUDA;
+  static SmemLimit lim;
+  cudaError_t e = allow_smem(gemm_swap_kernel, kSwSmem, lim);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ntiles * S, 1, 1);
+  cfg.blockDim = dim3(kSwThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSwSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gemm_swap_kernel, mA, a);
+  if (e != cudaSuccess) return cuda_fail(e);
+  HBL_CHECK_LAUNCH();
+  return HBL_OK;
+}
+
+// Token counts up to this bound run on CUDA cores when the codes come packed two per byte.
 constexpr int kDecodeMaxM = 8;
 // From this token count on, the product runs on SM pairs (256 x 256 tiles).
 constexpr int kPairMinM = 256;
@@ -306,7 +378,7 @@ hbl_status run_gemm(const void* codes, int fmt, int abits, const float* s_x, con
   const BlobLayout bl = blob_layout(K, N);
   const uint8_t* blob = static_cast<const uint8_t*>(packed);
   const bool packed4 = (abits == 4 && fmt == HBL_CODES_PACKED);
-  if (M <= kDecodeMaxM) {
+  if (packed4 && M <= kDecodeMaxM) {
     DecodeArgs d;
     d.m0 = 0;
     d.codes = static_cast<const uint8_t*>(codes);
@@ -332,8 +404,8 @@ hbl_status run_gemm(const void* codes, int fmt, int abits, const float* s_x, con
   t.Y = Y;
   t.out_bf16 = out_dtype == HBL_OUT_BF16;
   t.acc_debug = acc_debug;
-  const int8_t* w8 = reinterpret_cast<const int8_t*>(blob + bl.off1);
-  return M >= kPairMinM ? run_tc2(codes, w8, t, s) : run_tc(codes, w8, t, s);
+  if (M <= kSwapMaxM) return run_swap(codes, blob + bl.off0, t, s);
+  return run_tc2(codes, reinterpret_cast<const int8_t*>(blob + bl.off1), t, s);
 }
 
 size_t forward_codes_bytes(int M, int K) { return round_up((size_t)M * K, 256); }
@@ -488,7 +560,7 @@ hbl_status hbl_forward(const void* X, const float* gain, const void* packed, siz
   if (ws_bytes < hbl_forward_workspace(M, K, quant)) return HBL_EINVAL;
   if (packed_bytes < blob_layout(K, N).total || !aligned(packed, 256) || !aligned(Y, 16)) return HBL_EINVAL;
   const int abits = quant == HBL_Q_A8_ABSMAX ? 8 : 4;
-  const hbl_codes_fmt fmt = M <= kDecodeMaxM ? HBL_CODES_PACKED : HBL_CODES_I8;
+  const hbl_codes_fmt fmt = HBL_CODES_I8;  // both tensor-core products read one int8 per code
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* codes = ws;
   float* s_x = reinterpret_cast<float*>(ws + forward_codes_bytes(M, K));

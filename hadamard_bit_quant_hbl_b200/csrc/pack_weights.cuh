@@ -56,7 +56,10 @@ __global__ void __launch_bounds__(kAbsumThreads) absum_final_kernel(const double
 
 // One thread per (column n, 16-row group w): 16 ternary codes t[16w .. 16w+15][n].
 // Lanes take consecutive n, so every read of a W row segment is coalesced.
-//   section 0: uint32 word (n, w), code t+1 of k = 16w + 4s + b at bits 8b + 2s
+//   section 0: uint32 word (n, w), code t+1 of k = 16w + 4s + b at bits 8b + 2s, stored
+//              tile-major: word (n, w) at ((n/128) * (K/128) + w/8) * 1024 + (n%128) * 8 + w%8,
+//              so that one 128-feature x 128-k tile is 4 KB of contiguous memory. Rows of the
+//              last tile beyond N are filled with t = 0.
 //   section 1: int8 t[k][n] at n*K + k
 //   section 2: int32 column sum (atomic, integer: order-independent)
 template <bool FROM_CODES>
@@ -68,7 +71,11 @@ __global__ void __launch_bounds__(128) ternarize_pack_kernel(const float* __rest
                                                              int32_t* __restrict__ sec2) {
   const int n = blockIdx.x * 128 + threadIdx.x;
   const int w = blockIdx.y;
-  if (n >= N) return;
+  const size_t w2idx = ((size_t)(n >> 7) * (K >> 7) + (w >> 3)) * 1024 + (size_t)(n & 127) * 8 + (w & 7);
+  if (n >= N) {  // padding rows of the last 128-feature tile (section 0 only)
+    sec0[w2idx] = 0x55555555u;
+    return;
+  }
   int t[16];
   if constexpr (FROM_CODES) {
     bool bad = false;
@@ -106,7 +113,7 @@ __global__ void __launch_bounds__(128) ternarize_pack_kernel(const float* __rest
     b4[q] = ((uint32_t)(uint8_t)(int8_t)t[4 * q]) | ((uint32_t)(uint8_t)(int8_t)t[4 * q + 1] << 8) |
             ((uint32_t)(uint8_t)(int8_t)t[4 * q + 2] << 16) | ((uint32_t)(uint8_t)(int8_t)t[4 * q + 3] << 24);
   }
-  sec0[(size_t)n * (K / 16) + w] = word;
+  sec0[w2idx] = word;
   *reinterpret_cast<uint4*>(sec1 + (size_t)n * K + 16 * w) = make_uint4(b4[0], b4[1], b4[2], b4[3]);
   atomicAdd(sec2 + n, colsum);
 }

@@ -84,13 +84,16 @@ hbl_status hbl_device_status(hbl_stream_t stream);
  *
  * The packed blob (hbl_packed_weights_bytes(K, N) bytes, 256-byte aligned) holds, for the
  * logical K x N ternary matrix t:
- *   section 0 at byte 0:   2-bit codes, N rows of K/16 uint32 words (K-major). Word w of
- *                          row n holds t[16w + 4s + b][n] + 1 (in {0,1,2}) at bits 8b+2s
- *                          (b, s in 0..3). Read by the small-M (decode) product.
+ *   section 0 at byte 0:   2-bit codes as uint32 words: word w of feature n holds
+ *                          t[16w + 4s + b][n] + 1 (in {0,1,2}) at bits 8b+2s (b, s in 0..3).
+ *                          Words are tile-major: (n, w) is word number
+ *                          ((n/128)*(K/128) + w/8)*1024 + (n%128)*8 + w%8, so each 128-feature
+ *                          x 128-k tile is 4 KB of contiguous memory; features are padded to a
+ *                          multiple of 128 with t = 0. Read by the small-M products.
  *   section 1 at byte A1:  int8 t[k][n] as N rows of K bytes (K-major). Read by the
  *                          tensor-core product.
  *   section 2 at byte A2:  int32 column sums sum_k t[k][n], N entries.
- *   with A1 = round_up(N*K/4, 256), A2 = A1 + round_up(N*K, 256).
+ *   with A1 = round_up(round_up(N, 128)*K/4, 256), A2 = A1 + round_up(N*K, 256).
  * ------------------------------------------------------------------------------------- */
 size_t hbl_packed_weights_bytes(int K, int N);
 

@@ -28,7 +28,7 @@ def pack_int4(q: np.ndarray) -> np.ndarray:
 
 def blob_offsets(K: int, N: int):
     r = lambda v: (v + 255) // 256 * 256  # noqa: E731
-    off1 = r(N * K // 4)
+    off1 = r((N + 127) // 128 * 128 * K // 4)
     off2 = off1 + r(N * K)
     return 0, off1, off2, off2 + r(4 * N)
 
@@ -37,7 +37,10 @@ def decode_blob(blob: np.ndarray, K: int, N: int):
     """Packed weight blob -> (t from the 2-bit section [K, N], t from the int8 section [K, N], column sums)."""
     o0, o1, o2, _ = blob_offsets(K, N)
     b = np.asarray(blob, dtype=np.uint8)
-    words = b[o0:o0 + N * K // 4].view(np.uint32).reshape(N, K // 16)
+    NP = (N + 127) // 128 * 128
+    # tile-major: [N/128 tiles][K/128 blocks][128 rows][8 words] -> [NP rows][K/16 words]
+    tiles = b[o0:o0 + NP * K // 4].view(np.uint32).reshape(NP // 128, K // 128, 128, 8)
+    words = tiles.transpose(0, 2, 1, 3).reshape(NP, K // 16)[:N]
     t2 = np.empty((N, K), dtype=np.int8)
     for s in range(4):
         for bb in range(4):

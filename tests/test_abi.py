@@ -45,7 +45,8 @@ def test_status_strings(L):
 def test_sizes(L):
     K, N = 4096, 2560
     r = lambda v: (v + 255) // 256 * 256  # noqa: E731
-    assert hbl.hbl_packed_weights_bytes(K, N) == r(N * K // 4) + r(N * K) + r(4 * N)
+    assert hbl.hbl_packed_weights_bytes(K, N) == r(N * K // 4) + r(N * K) + r(4 * N)  # N a multiple of 128
+    assert hbl.hbl_packed_weights_bytes(K, 520) == r(640 * K // 4) + r(520 * K) + r(4 * 520)
     assert hbl.hbl_packed_weights_bytes(0, N) == 0
     assert hbl.hbl_forward_workspace(100, 4096, hbl.HBL_Q_A4_ABSMEAN) == r(100 * 4096) + r(400)
     assert hbl.hbl_pack_weights_workspace(K, N) >= 8 * 593
