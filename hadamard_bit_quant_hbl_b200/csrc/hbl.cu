@@ -108,8 +108,7 @@ hbl_status launch_nfq_t(const NfqArgs& a, int threads, int smem, cudaStream_t s)
   auto* k = norm_fht_quant_kernel<L, EB, R, G, QM>;
   const cudaError_t e = allow_smem(k, smem, lim);
   if (e != cudaSuccess) return cuda_fail(e);
-  const int grid = persistent_grid(k, threads, smem, a.groups);
-  k<<<grid, threads, smem, s>>>(a);
+  k<<<a.groups, threads, smem, s>>>(a);
   HBL_CHECK_LAUNCH();
   return HBL_OK;
 }
@@ -140,11 +139,9 @@ hbl_status run_nfq(const void* X, const float* gain, int M, int K, int had_block
   const int nb = K / n;
   int R = 1, slots = 1, rows = 1;
   if (nb == 1) {
-    // a group of rows per CTA: about 256 threads and <= 96 KB of shared memory (bf16 landing
-    // buffer + fp32 regrouping buffer), so that two CTAs fit on an SM
-    rows = 256 / P;
-    const int cap = (96 * 1024) / (K * 6);
-    if (rows > cap) rows = cap;
+    // a group of rows per CTA: about 128 threads and <= 64 KB of fp32 regrouping buffer, so that
+    // three or more CTAs fit on an SM
+    rows = 128 / P;
     if (rows < 1) rows = 1;
     if (P == 16 && rows > 1 && (rows & 1)) rows -= 1;  // half-warp rows come in pairs
   } else {
@@ -159,7 +156,7 @@ hbl_status run_nfq(const void* X, const float* gain, int M, int K, int had_block
     if (slots * P > maxt) return HBL_EUNSUPPORTED;
   }
   const int threads = rows * slots * P;
-  const int smem = rows * K * 6;
+  const int smem = rows * K * 4;
 
   NfqArgs a;
   a.X = static_cast<const uint16_t*>(X);

@@ -4,14 +4,14 @@
 // applies an online Hadamard transform, computed with the fast Hadamard transform in
 // O(n log n), to the normalised activations before quantising them per token to INT8 or INT4.
 //
-// The kernel is persistent: a CTA owns a group of `rows` token rows at a time and walks over
-// the groups; while it transforms one group, the TMA engine copies the next group's bf16 rows
-// into shared memory (one 1-D bulk copy, completion on an mbarrier).
+// A CTA owns `rows` token rows (one row for the big transforms). Its threads load the bf16
+// row straight from global memory into registers; several CTAs share an SM, so that one CTA's
+// loads are in flight while the others compute.
 //
 // One token row has K = nb blocks of n = 2^L features (nb = 1 for a transform over all of K).
 // A block is transformed by P = 2^(L-EB) threads holding E = 2^EB values each:
 //   1. "layout 1": a thread holds 8 consecutive features (index bits 0..2) for each of the
-//      2^(EB-3) top index bits; read from the landing buffer as 16-byte vectors; the sum of
+//      2^(EB-3) top index bits; read from global memory as 16-byte vectors; the sum of
 //      squares for the RMS accumulates here; all EB butterfly stages run in registers.
 //   2. one pass through shared memory (128-bit stores, scalar loads, XOR swizzle checked at
 //      compile time) regroups the values so that index bits 3..TOP-1 are in registers
@@ -162,25 +162,35 @@ __device__ __forceinline__ void fwht_regs2(float2 (&v)[E / 2]) {
 
 // ---------------------------------------------------------------- the kernel
 
-// Largest CTA a plan is launched with (bounds the register budget of the big transforms).
+// Largest CTA a plan is launched with, and the register cap that lets several such CTAs share
+// an SM (the big transforms hold 128 values per thread).
 constexpr int nfq_max_threads(int L) { return L >= 11 ? 256 : 512; }
+constexpr int nfq_max_regs(int EB, int R) {
+  return ((1 << EB) * R) >= 128 ? 168 : (((1 << EB) * R) >= 64 ? 128 : 96);
+}
+
+// 16-byte streaming load that bypasses L1 (every input byte is read once).
+__device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
 
 // QM: 0 = a8 absmax, 1 = a4 absmean, 2 = a4 absmax
 template <int L, int EB, int R, bool HAS_GAIN, int QM>
-__global__ void __launch_bounds__(nfq_max_threads(L)) norm_fht_quant_kernel(const NfqArgs a) {
+__global__ void __maxnreg__(nfq_max_regs(EB, R)) norm_fht_quant_kernel(const NfqArgs a) {
   using Pl = FhtPlan<L, EB>;
   static_assert(Pl::check_store1(), "layout-1 stores have bank conflicts");
   static_assert(Pl::load2_ways() <= (Pl::XB ? 2 : 1), "layout-2 loads have avoidable bank conflicts");
   constexpr int n = Pl::n, P = Pl::P, E = Pl::E, NV = Pl::NV, S2 = Pl::S2, XB = Pl::XB;
   extern __shared__ __align__(128) uint8_t smem_nfq[];
   __shared__ float red_ss[32], red_st[32];
-  __shared__ __align__(8) uint64_t land_bar;
-  __shared__ volatile int abort_flag;
 
   const int K = a.K, nb = a.nb, rows = a.rows;
-  uint16_t* land = reinterpret_cast<uint16_t*>(smem_nfq);                   // rows*K bf16
-  float* fbuf = reinterpret_cast<float*>(smem_nfq + (size_t)rows * K * 2);  // rows*K fp32
-  uint8_t* cbuf = reinterpret_cast<uint8_t*>(fbuf);                         // codes, aliases fbuf
+  float* fbuf = reinterpret_cast<float*>(smem_nfq);  // rows*K fp32 (regrouping)
+  uint8_t* cbuf = smem_nfq;                          // codes, reuses the regrouping buffer
   const int crow = K / 8 + 16;  // byte stride of one (k mod 8) row of the code matrix (padded)
 
   const int tid = threadIdx.x;
@@ -190,58 +200,41 @@ __global__ void __launch_bounds__(nfq_max_threads(L)) norm_fht_quant_kernel(cons
   const int slot = tr / P;
   const int pt = tr - slot * P;
   const int lane = tid & 31, warp = tid >> 5;
+  const int g = blockIdx.x;
+  const int row = g * rows + rloc;
+  const bool live_row = row < a.M;
 
   constexpr float kQ = QM == 0 ? 127.f : (QM == 1 ? 2.6457513110645906f : 7.f);
   constexpr int kLo = QM == 0 ? -128 : -8, kHi = QM == 0 ? 127 : 7;
   constexpr bool kAbsmax = QM != 1;
 
-  if (tid == 0) {
-    abort_flag = 0;
-    mbar_init(&land_bar, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncthreads();
-
-  int g = blockIdx.x;
-  if (tid == 0 && g < a.groups) {
-    const int nr = min(rows, a.M - g * rows);
-    const uint32_t bytes = (uint32_t)nr * (uint32_t)K * 2u;
-    mbar_arrive_expect_tx(&land_bar, bytes);
-    bulk_load_1d(land, a.X + (size_t)g * rows * K, bytes, &land_bar);
-  }
-  bool pending = g < a.groups;
-  uint32_t phase = 0;
-
-  for (; g < a.groups; g += gridDim.x) {
-    const int row = g * rows + rloc;
-    const bool live_row = row < a.M;
-
-    // ---- wait for this group's rows (every thread; bounded)
-    if (!mbar_wait(&land_bar, phase, &abort_flag)) abort_flag = 1;
-    __syncthreads();
-    if (abort_flag) break;
-    phase ^= 1u;
-    pending = false;
-
-    // ---- 1. layout 1 from the landing buffer, sum of squares (+ gain)
-    float2 v[R][E / 2];
-    float2 ss2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  // ---- 1. layout 1 straight from global memory (16-byte vectors, every load issued before the
+  // first use), sum of squares (+ gain)
+  float2 v[R][E / 2];
+  float2 ss2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  {
+    uint4 w[R][NV];
 #pragma unroll
     for (int rho = 0; rho < R; ++rho) {
       const int blk = slot + rho * a.slots;
       const bool live = live_row && blk < nb;
-      const uint16_t* src = land + (size_t)rloc * K + (size_t)blk * n + (pt << 3);
+      const uint16_t* src = a.X + (size_t)row * K + (size_t)blk * n + (pt << 3);
+#pragma unroll
+      for (int vv = 0; vv < NV; ++vv) w[rho][vv] = live ? ldg_stream_v4(src + (vv << Pl::TOP)) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int rho = 0; rho < R; ++rho) {
+      const int blk = slot + rho * a.slots;
 #pragma unroll
       for (int vv = 0; vv < NV; ++vv) {
-        uint4 w = make_uint4(0u, 0u, 0u, 0u);
-        if (live) w = *reinterpret_cast<const uint4*>(src + (vv << Pl::TOP));
-        const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+        const uint32_t u[4] = {w[rho][vv].x, w[rho][vv].y, w[rho][vv].z, w[rho][vv].w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          float2 f = make_float2(__uint_as_float(u[i] << 16), __uint_as_float(u[i] & 0xffff0000u));
+          // bf16 -> fp32 on the integer/logic units: low half moved up by a byte permute
+          float2 f = make_float2(__uint_as_float(__byte_perm(u[i], 0u, 0x1044)), __uint_as_float(u[i] & 0xffff0000u));
           ss2[i] = __ffma2_rn(f, f, ss2[i]);  // independent chains
           if constexpr (HAS_GAIN) {
-            if (live) {
+            if (live_row && blk < nb) {
               const float2 gg = *reinterpret_cast<const float2*>(a.gain + (size_t)blk * n + (vv << Pl::TOP) +
                                                                  (pt << 3) + 2 * i);
               f = __fmul2_rn(f, gg);
@@ -251,210 +244,201 @@ __global__ void __launch_bounds__(nfq_max_threads(L)) norm_fht_quant_kernel(cons
         }
       }
     }
-    __syncthreads();  // landing buffer consumed: prefetch the next group
-    const int gn = g + (int)gridDim.x;
-    if (tid == 0 && gn < a.groups) {
-      const int nr = min(rows, a.M - gn * rows);
-      const uint32_t bytes = (uint32_t)nr * (uint32_t)K * 2u;
-      mbar_arrive_expect_tx(&land_bar, bytes);
-      bulk_load_1d(land, a.X + (size_t)gn * rows * K, bytes, &land_bar);
-    }
-    pending = gn < a.groups;
-    float ss = ((ss2[0].x + ss2[0].y) + (ss2[1].x + ss2[1].y)) + ((ss2[2].x + ss2[2].y) + (ss2[3].x + ss2[3].y));
+  }
+  float ss = ((ss2[0].x + ss2[0].y) + (ss2[1].x + ss2[1].y)) + ((ss2[2].x + ss2[2].y) + (ss2[3].x + ss2[3].y));
 
 #pragma unroll
-    for (int rho = 0; rho < R; ++rho) fwht_regs2<E, EB>(v[rho]);
+  for (int rho = 0; rho < R; ++rho) fwht_regs2<E, EB>(v[rho]);
 
-    // ---- 2. regroup through shared memory (index within the CTA buffer: (rloc*nb + blk)*n + i)
-    const uint32_t rowbase = (uint32_t)rloc * (uint32_t)K;
+  // ---- 2. regroup through shared memory (index within the CTA buffer: (rloc*nb + blk)*n + i)
+  const uint32_t rowbase = (uint32_t)rloc * (uint32_t)K;
 #pragma unroll
-    for (int rho = 0; rho < R; ++rho) {
-      const int blk = slot + rho * a.slots;
-      if (blk < nb) {
-        const SwzBases<Pl> sb(rowbase + ((uint32_t)blk << L) + ((uint32_t)pt << 3));
+  for (int rho = 0; rho < R; ++rho) {
+    const int blk = slot + rho * a.slots;
+    if (blk < nb) {
+      const SwzBases<Pl> sb(rowbase + ((uint32_t)blk << L) + ((uint32_t)pt << 3));
 #pragma unroll
-        for (int r = 0; r < E; r += 4) {
-          const float4 q4 = make_float4(v[rho][r / 2].x, v[rho][r / 2].y, v[rho][r / 2 + 1].x, v[rho][r / 2 + 1].y);
-          *reinterpret_cast<float4*>(fbuf + sb.at((uint32_t)Pl::idx1(0, r))) = q4;
-        }
+      for (int r = 0; r < E; r += 4) {
+        const float4 q4 = make_float4(v[rho][r / 2].x, v[rho][r / 2].y, v[rho][r / 2 + 1].x, v[rho][r / 2 + 1].y);
+        *reinterpret_cast<float4*>(fbuf + sb.at((uint32_t)Pl::idx1(0, r))) = q4;
       }
     }
-    __syncthreads();
+  }
+  __syncthreads();
 #pragma unroll
-    for (int rho = 0; rho < R; ++rho) {
-      const int blk = slot + rho * a.slots;
-      if (blk < nb) {
-        const SwzBases<Pl> sb(rowbase + ((uint32_t)blk << L) + (uint32_t)Pl::idx2(pt, 0));
+  for (int rho = 0; rho < R; ++rho) {
+    const int blk = slot + rho * a.slots;
+    if (blk < nb) {
+      const SwzBases<Pl> sb(rowbase + ((uint32_t)blk << L) + (uint32_t)Pl::idx2(pt, 0));
 #pragma unroll
-        for (int r = 0; r < E; r += 2) {
-          v[rho][r / 2].x = fbuf[sb.at((uint32_t)Pl::idx2(0, r))];
-          v[rho][r / 2].y = fbuf[sb.at((uint32_t)Pl::idx2(0, r + 1))];
-        }
-        fwht_regs2<E, S2>(v[rho]);
-      } else {
-#pragma unroll
-        for (int r = 0; r < E / 2; ++r) v[rho][r] = make_float2(0.f, 0.f);
+      for (int r = 0; r < E; r += 2) {
+        v[rho][r / 2].x = fbuf[sb.at((uint32_t)Pl::idx2(0, r))];
+        v[rho][r / 2].y = fbuf[sb.at((uint32_t)Pl::idx2(0, r + 1))];
       }
-    }
-
-    // ---- 3. row statistics
-    float sta[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent chains
-#pragma unroll
-    for (int rho = 0; rho < R; ++rho) {
-#pragma unroll
-      for (int r = 0; r < E / 2; ++r) {
-        float& acc = sta[(rho * (E / 2) + r) & 7];
-        if constexpr (kAbsmax) acc = fmaxf(acc, fmaxf(fabsf(v[rho][r].x), fabsf(v[rho][r].y)));
-        else acc += fabsf(v[rho][r].x) + fabsf(v[rho][r].y);
-      }
-    }
-    float st;
-    if constexpr (kAbsmax) {
-      st = fmaxf(fmaxf(fmaxf(sta[0], sta[1]), fmaxf(sta[2], sta[3])), fmaxf(fmaxf(sta[4], sta[5]), fmaxf(sta[6], sta[7])));
+      fwht_regs2<E, S2>(v[rho]);
     } else {
-      st = ((sta[0] + sta[1]) + (sta[2] + sta[3])) + ((sta[4] + sta[5]) + (sta[6] + sta[7]));
+#pragma unroll
+      for (int r = 0; r < E / 2; ++r) v[rho][r] = make_float2(0.f, 0.f);
     }
-    if (tpr >= 32) {
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) {
-        ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        const float t = __shfl_xor_sync(0xffffffffu, st, o);
-        st = kAbsmax ? fmaxf(st, t) : st + t;
-      }
-      if (lane == 0) {
-        red_ss[warp] = ss;
-        red_st[warp] = st;
-      }
-      __syncthreads();
-      const int w0 = (rloc * tpr) >> 5, nw = tpr >> 5;
-      ss = 0.f;
-      st = 0.f;
-      for (int w = 0; w < nw; ++w) {  // fixed order: the same result in every thread of the row
-        ss += red_ss[w0 + w];
-        st = kAbsmax ? fmaxf(st, red_st[w0 + w]) : st + red_st[w0 + w];
-      }
-    } else {  // 16 threads per row, two rows per warp
-#pragma unroll
-      for (int o = 8; o >= 1; o >>= 1) {
-        ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        const float t = __shfl_xor_sync(0xffffffffu, st, o);
-        st = kAbsmax ? fmaxf(st, t) : st + t;
-      }
-      __syncthreads();  // every layout-2 read is done before codes overwrite the buffer
-    }
-
-    // ---- 4. per-row multiplier and scale
-    const float r_rms = sqrtf(ss / (float)K + a.eps_norm);
-    const float rs = r_rms * sqrtf((float)n);        // y = xr * rs (xr = orthonormal output)
-    const float sy = kAbsmax ? st : st / (float)K;  // statistic of y
-    float mult, sx;
-    if (a.eps_q == 0.f) {
-      mult = sy > 0.f ? kQ / sy : 0.f;
-      sx = sy > 0.f ? sy / (rs * kQ) : 0.f;
-    } else {
-      const float stat = sy / rs;                     // statistic of xr
-      mult = kQ / ((stat + a.eps_q) * rs);
-      sx = stat / kQ;
-    }
-    if (live_row && tr == 0) a.s_x[row] = sx;
-
-    // ---- 5. codes: fp32 product, clamp (absmean only: absmax products already lie in
-    // [-Q, Q]), then round to nearest even by adding 1.5 * 2^23 -- the integer lands in the low
-    // mantissa bits and, being small, its low 16 bits are the int16 code. 4 codes per word,
-    // 16 bytes per store.
-    const float2 mult2 = make_float2(mult, mult);
-    const float2 magic2 = make_float2(12582912.f, 12582912.f);
-#pragma unroll
-    for (int rho = 0; rho < R; ++rho) {
-      const int blk = slot + rho * a.slots;
-      if (blk < nb) {
-#pragma unroll
-        for (int x = 0; x < (1 << XB); ++x) {
-          // codes of registers r = (x << S2) | j are those of k = 8 * (c0 + j) + b
-          const int b = x | ((pt & ((1 << (3 - XB)) - 1)) << XB);
-          const int c0 = (blk << (L - 3)) + ((pt >> (3 - XB)) << (Pl::TOP - 3));
-          uint8_t* dst = cbuf + (size_t)rloc * 8 * crow + (size_t)b * crow + c0;
-#pragma unroll
-          for (int j = 0; j < (1 << S2); j += 16) {
-            uint32_t wds[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int r0 = (x << S2) + j + 4 * q;  // 4 consecutive registers = 2 float2
-              float2 t0 = __fmul2_rn(v[rho][r0 / 2], mult2);
-              float2 t1 = __fmul2_rn(v[rho][r0 / 2 + 1], mult2);
-              if constexpr (!kAbsmax) {
-                t0.x = fminf(fmaxf(t0.x, (float)kLo), (float)kHi);
-                t0.y = fminf(fmaxf(t0.y, (float)kLo), (float)kHi);
-                t1.x = fminf(fmaxf(t1.x, (float)kLo), (float)kHi);
-                t1.y = fminf(fmaxf(t1.y, (float)kLo), (float)kHi);
-              }
-              const float2 p0 = __fadd2_rn(t0, magic2);
-              const float2 p1 = __fadd2_rn(t1, magic2);
-              const uint32_t h0 = __byte_perm(__float_as_uint(p0.x), __float_as_uint(p0.y), 0x5410);
-              const uint32_t h1 = __byte_perm(__float_as_uint(p1.x), __float_as_uint(p1.y), 0x5410);
-              wds[q] = __byte_perm(h0, h1, 0x6420);
-            }
-            *reinterpret_cast<uint4*>(dst + j) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
-          }
-        }
-      }
-    }
-    __syncthreads();
-
-    // ---- 6. stream codes out in natural order, 32 consecutive codes per unit
-    const int upr = K / 32;  // units per row
-    const bool packed4 = (a.fmt == 0) && (QM != 0);
-    // thread tid handles units tid, tid + blockDim, ... of the CTA's rows * upr units; walk them
-    // row by row without dividing
-    int rl = 0, vcol = tid;
-    while (vcol >= upr && rl < rows) { vcol -= upr; ++rl; }
-    for (; rl < rows; vcol += blockDim.x) {
-      while (vcol >= upr) { vcol -= upr; ++rl; }
-      if (rl >= rows) break;
-      const int grow = g * rows + rl;
-      if (grow >= a.M) continue;
-      const uint8_t* srcc = cbuf + (size_t)rl * 8 * crow + 4 * vcol;
-      uint32_t w[8];
-#pragma unroll
-      for (int b = 0; b < 8; ++b) w[b] = *reinterpret_cast<const uint32_t*>(srcc + (size_t)b * crow);
-      // byte j of w[b] is the code of k = 32 * vcol + 8 * j + b
-      if (!packed4) {
-        uint32_t o[8];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {  // k mod 8 = 4h .. 4h+3
-          const uint32_t a01l = __byte_perm(w[4 * h], w[4 * h + 1], 0x5140);
-          const uint32_t a01h = __byte_perm(w[4 * h], w[4 * h + 1], 0x7362);
-          const uint32_t a23l = __byte_perm(w[4 * h + 2], w[4 * h + 3], 0x5140);
-          const uint32_t a23h = __byte_perm(w[4 * h + 2], w[4 * h + 3], 0x7362);
-          o[0 + h] = __byte_perm(a01l, a23l, 0x5410);  // j = 0
-          o[2 + h] = __byte_perm(a01l, a23l, 0x7632);  // j = 1
-          o[4 + h] = __byte_perm(a01h, a23h, 0x5410);  // j = 2
-          o[6 + h] = __byte_perm(a01h, a23h, 0x7632);  // j = 3
-        }
-        uint4* dstg = reinterpret_cast<uint4*>(a.codes + (size_t)grow * K + 32 * vcol);
-        dstg[0] = make_uint4(o[0], o[1], o[2], o[3]);
-        dstg[1] = make_uint4(o[4], o[5], o[6], o[7]);
-      } else {
-        // nibble pairs first: byte j of m[i] = code(8j + 2i) | code(8j + 2i + 1) << 4
-        uint32_t m[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) m[i] = (w[2 * i] & 0x0f0f0f0fu) | ((w[2 * i + 1] & 0x0f0f0f0fu) << 4);
-        const uint32_t a01l = __byte_perm(m[0], m[1], 0x5140);
-        const uint32_t a01h = __byte_perm(m[0], m[1], 0x7362);
-        const uint32_t a23l = __byte_perm(m[2], m[3], 0x5140);
-        const uint32_t a23h = __byte_perm(m[2], m[3], 0x7362);
-        const uint4 o = make_uint4(__byte_perm(a01l, a23l, 0x5410), __byte_perm(a01l, a23l, 0x7632),
-                                   __byte_perm(a01h, a23h, 0x5410), __byte_perm(a01h, a23h, 0x7632));
-        *reinterpret_cast<uint4*>(a.codes + (size_t)grow * (K / 2) + 16 * vcol) = o;
-      }
-    }
-    // the next iteration's first __syncthreads orders these reads before the buffer is rewritten
   }
 
-  // an early exit must not leave a copy in flight into shared memory
-  if (tid == 0 && pending) {
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(&land_bar, phase) && globaltimer_ns() - t0 < kWaitLimitNs) {
+  // ---- 3. row statistics: sum |y| as pairwise sums folded into fp32x2 chains, or max |y|
+  float st;
+  if constexpr (kAbsmax) {
+    float sta[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int rho = 0; rho < R; ++rho)
+#pragma unroll
+      for (int r = 0; r < E / 2; ++r) {
+        float& acc = sta[(rho * (E / 2) + r) & 3];
+        acc = fmaxf(acc, fmaxf(fabsf(v[rho][r].x), fabsf(v[rho][r].y)));
+      }
+    st = fmaxf(fmaxf(sta[0], sta[1]), fmaxf(sta[2], sta[3]));
+  } else {
+    float2 sta2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+    for (int rho = 0; rho < R; ++rho)
+#pragma unroll
+      for (int r = 0; r < E / 2; r += 2) {
+        const float2 t = make_float2(fabsf(v[rho][r].x) + fabsf(v[rho][r].y),
+                                     fabsf(v[rho][r + 1].x) + fabsf(v[rho][r + 1].y));
+        float2& acc = sta2[(rho * (E / 4) + r / 2) & 3];
+        acc = __fadd2_rn(acc, t);
+      }
+    st = ((sta2[0].x + sta2[0].y) + (sta2[1].x + sta2[1].y)) + ((sta2[2].x + sta2[2].y) + (sta2[3].x + sta2[3].y));
+  }
+  if (tpr >= 32) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float t = __shfl_xor_sync(0xffffffffu, st, o);
+      st = kAbsmax ? fmaxf(st, t) : st + t;
+    }
+    if (lane == 0) {
+      red_ss[warp] = ss;
+      red_st[warp] = st;
+    }
+    __syncthreads();  // also: every layout-2 read is done before codes overwrite the buffer
+    const int w0 = (rloc * tpr) >> 5, nw = tpr >> 5;
+    ss = 0.f;
+    st = 0.f;
+    for (int w = 0; w < nw; ++w) {  // fixed order: the same result in every thread of the row
+      ss += red_ss[w0 + w];
+      st = kAbsmax ? fmaxf(st, red_st[w0 + w]) : st + red_st[w0 + w];
+    }
+  } else {  // 16 threads per row, two rows per warp
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) {
+      ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float t = __shfl_xor_sync(0xffffffffu, st, o);
+      st = kAbsmax ? fmaxf(st, t) : st + t;
+    }
+    __syncthreads();  // every layout-2 read is done before codes overwrite the buffer
+  }
+
+  // ---- 4. per-row multiplier and scale
+  const float r_rms = sqrtf(ss / (float)K + a.eps_norm);
+  const float rs = r_rms * sqrtf((float)n);        // y = xr * rs (xr = orthonormal output)
+  const float sy = kAbsmax ? st : st / (float)K;  // statistic of y
+  float mult, sx;
+  if (a.eps_q == 0.f) {
+    mult = sy > 0.f ? kQ / sy : 0.f;
+    sx = sy > 0.f ? sy / (rs * kQ) : 0.f;
+  } else {
+    const float stat = sy / rs;                     // statistic of xr
+    mult = kQ / ((stat + a.eps_q) * rs);
+    sx = stat / kQ;
+  }
+  if (live_row && tr == 0) a.s_x[row] = sx;
+
+  // ---- 5. codes: fp32 product, clamp (absmean only: absmax products already lie in
+  // [-Q, Q]), then round to nearest even by adding 1.5 * 2^23 -- the integer lands in the low
+  // mantissa bits and, being small, its low 16 bits are the int16 code. 4 codes per word,
+  // 16 bytes per store, into a byte matrix [k mod 8][k / 8].
+  const float2 mult2 = make_float2(mult, mult);
+  const float2 magic2 = make_float2(12582912.f, 12582912.f);
+#pragma unroll
+  for (int rho = 0; rho < R; ++rho) {
+    const int blk = slot + rho * a.slots;
+    if (blk < nb) {
+#pragma unroll
+      for (int x = 0; x < (1 << XB); ++x) {
+        // codes of registers r = (x << S2) | j are those of k = 8 * (c0 + j) + b
+        const int b = x | ((pt & ((1 << (3 - XB)) - 1)) << XB);
+        const int c0 = (blk << (L - 3)) + ((pt >> (3 - XB)) << (Pl::TOP - 3));
+        uint8_t* dst = cbuf + (size_t)rloc * 8 * crow + (size_t)b * crow + c0;
+#pragma unroll
+        for (int j = 0; j < (1 << S2); j += 16) {
+          uint32_t wds[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int r0 = (x << S2) + j + 4 * q;  // 4 consecutive registers = 2 float2
+            float2 t0 = __fmul2_rn(v[rho][r0 / 2], mult2);
+            float2 t1 = __fmul2_rn(v[rho][r0 / 2 + 1], mult2);
+            if constexpr (!kAbsmax) {
+              t0.x = fminf(fmaxf(t0.x, (float)kLo), (float)kHi);
+              t0.y = fminf(fmaxf(t0.y, (float)kLo), (float)kHi);
+              t1.x = fminf(fmaxf(t1.x, (float)kLo), (float)kHi);
+              t1.y = fminf(fmaxf(t1.y, (float)kLo), (float)kHi);
+            }
+            const float2 p0 = __fadd2_rn(t0, magic2);
+            const float2 p1 = __fadd2_rn(t1, magic2);
+            const uint32_t h0 = __byte_perm(__float_as_uint(p0.x), __float_as_uint(p0.y), 0x5410);
+            const uint32_t h1 = __byte_perm(__float_as_uint(p1.x), __float_as_uint(p1.y), 0x5410);
+            wds[q] = __byte_perm(h0, h1, 0x6420);
+          }
+          *reinterpret_cast<uint4*>(dst + j) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- 6. stream codes out in natural order, 32 consecutive codes per unit
+  const int upr = K / 32;  // units per row
+  const bool packed4 = (a.fmt == 0) && (QM != 0);
+  // thread tid handles units tid, tid + blockDim, ... of the CTA's rows * upr units; walk them
+  // row by row without dividing
+  int rl = 0, vcol = tid;
+  while (vcol >= upr && rl < rows) { vcol -= upr; ++rl; }
+  for (; rl < rows; vcol += blockDim.x) {
+    while (vcol >= upr) { vcol -= upr; ++rl; }
+    if (rl >= rows) break;
+    const int grow = g * rows + rl;
+    if (grow >= a.M) break;  // rows past M are the CTA's last ones
+    const uint8_t* srcc = cbuf + (size_t)rl * 8 * crow + 4 * vcol;
+    uint32_t w[8];
+#pragma unroll
+    for (int b = 0; b < 8; ++b) w[b] = *reinterpret_cast<const uint32_t*>(srcc + (size_t)b * crow);
+    // byte j of w[b] is the code of k = 32 * vcol + 8 * j + b
+    if (!packed4) {
+      uint32_t o[8];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {  // k mod 8 = 4h .. 4h+3
+        const uint32_t a01l = __byte_perm(w[4 * h], w[4 * h + 1], 0x5140);
+        const uint32_t a01h = __byte_perm(w[4 * h], w[4 * h + 1], 0x7362);
+        const uint32_t a23l = __byte_perm(w[4 * h + 2], w[4 * h + 3], 0x5140);
+        const uint32_t a23h = __byte_perm(w[4 * h + 2], w[4 * h + 3], 0x7362);
+        o[0 + h] = __byte_perm(a01l, a23l, 0x5410);  // j = 0
+        o[2 + h] = __byte_perm(a01l, a23l, 0x7632);  // j = 1
+        o[4 + h] = __byte_perm(a01h, a23h, 0x5410);  // j = 2
+        o[6 + h] = __byte_perm(a01h, a23h, 0x7632);  // j = 3
+      }
+      uint4* dstg = reinterpret_cast<uint4*>(a.codes + (size_t)grow * K + 32 * vcol);
+      dstg[0] = make_uint4(o[0], o[1], o[2], o[3]);
+      dstg[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    } else {
+      // nibble pairs first: byte j of m[i] = code(8j + 2i) | code(8j + 2i + 1) << 4
+      uint32_t m[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) m[i] = (w[2 * i] & 0x0f0f0f0fu) | ((w[2 * i + 1] & 0x0f0f0f0fu) << 4);
+      const uint32_t a01l = __byte_perm(m[0], m[1], 0x5140);
+      const uint32_t a01h = __byte_perm(m[0], m[1], 0x7362);
+      const uint32_t a23l = __byte_perm(m[2], m[3], 0x5140);
+      const uint32_t a23h = __byte_perm(m[2], m[3], 0x7362);
+      const uint4 o = make_uint4(__byte_perm(a01l, a23l, 0x5410), __byte_perm(a01l, a23l, 0x7632),
+                                 __byte_perm(a01h, a23h, 0x5410), __byte_perm(a01h, a23h, 0x7632));
+      *reinterpret_cast<uint4*>(a.codes + (size_t)grow * (K / 2) + 16 * vcol) = o;
     }
   }
 }
