@@ -108,7 +108,11 @@ hbl_status launch_nfq_t(const NfqArgs& a, int threads, int smem, cudaStream_t s)
   auto* k = norm_fht_quant_kernel<L, EB, R, G, QM>;
   const cudaError_t e = allow_smem(k, smem, lim);
   if (e != cudaSuccess) return cuda_fail(e);
-  k<<<a.groups, threads, smem, s>>>(a);
+  NfqArgs b = a;
+  // prefetch distance: the groups resident on the device at once (the group that starts when
+  // this CTA's successor does)
+  b.pf_dist = persistent_grid(k, threads, smem, 1 << 30);
+  k<<<b.groups, threads, smem, s>>>(b);
   HBL_CHECK_LAUNCH();
   return HBL_OK;
 }
@@ -172,6 +176,7 @@ hbl_status run_nfq(const void* X, const float* gain, int M, int K, int had_block
   a.slots = slots;
   a.rows = rows;
   a.groups = (M + rows - 1) / rows;
+  a.pf_dist = 0;
 
   // K <= 32768 bounds nb, so these R always suffice: L=8 nb<=128 (R<=4), L=9..12 R<=2, L>=13 R=1
   switch (L) {
@@ -195,26 +200,59 @@ hbl_status run_nfq(const void* X, const float* gain, int M, int K, int had_block
 
 // ---------------------------------------------------------------- products
 
-template <int MT, int COLS>
-hbl_status launch_decode_t(const DecodeArgs& a, cudaStream_t s) {
-  const int units = a.K / 64;
-  const int threads = (units + 31) / 32 * 32;
-  const int grid = (a.N + COLS - 1) / COLS;
-  gemm_decode_kernel<MT, COLS><<<grid, threads, 0, s>>>(a);
+template <int MT>
+hbl_status launch_decode_t(const DecodeArgs& a, int smem, cudaStream_t s) {
+  static SmemLimit lim;
+  cudaError_t e = allow_smem(gemm_decode_kernel<MT>, smem, lim);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(((a.N + 127) / 128) * a.S, 1, 1);
+  cfg.blockDim = dim3(kDecThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = a.S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gemm_decode_kernel<MT>, a);
+  if (e != cudaSuccess) return cuda_fail(e);
   HBL_CHECK_LAUNCH();
   return HBL_OK;
 }
 
-// Rows are handled MT at a time (one launch per slice of MT rows).
+// One launch per slice of up to 8 token rows. A cluster of S CTAs splits K for each 128-feature
+// tile: S is chosen so that about two CTAs run per SM, and large enough that the CTA's staged
+// activations stay within 64 KB.
 hbl_status run_decode(const DecodeArgs& a0, cudaStream_t s) {
   DecodeArgs a = a0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int ntiles = (a.N + 127) / 128;
+  const int KB = a.K / 128;
   for (a.m0 = 0; a.m0 < a0.M;) {
     const int left = a0.M - a.m0;
+    const int MT = left == 1 ? 1 : left == 2 ? 2 : left <= 4 ? 4 : 8;
+    int S = (2 * device_sms(dev) + ntiles - 1) / ntiles;
+    const int smin = (a.K * MT + 65535) / 65536;
+    if (S < smin) S = smin;
+    if (S > 8) S = 8;
+    if (S > KB) S = KB;
+    if (S < 1) S = 1;
+    a.S = S;
+    const int range = (KB + S - 1) / S * 128;
+    const int smem = MT * range + MT * 128 * 4;
     hbl_status st;
-    if (left == 1) { st = launch_decode_t<1, 16>(a, s); a.m0 += 1; }
-    else if (left == 2) { st = launch_decode_t<2, 8>(a, s); a.m0 += 2; }
-    else { st = launch_decode_t<4, 4>(a, s); a.m0 += 4; }
+    switch (MT) {
+      case 1: st = launch_decode_t<1>(a, smem, s); break;
+      case 2: st = launch_decode_t<2>(a, smem, s); break;
+      case 4: st = launch_decode_t<4>(a, smem, s); break;
+      default: st = launch_decode_t<8>(a, smem, s); break;
+    }
     if (st != HBL_OK) return st;
+    a.m0 += MT;
   }
   return HBL_OK;
 }
@@ -365,7 +403,7 @@ hbl_status run_swap(const void* codes_i8, const void* w2, const TcArgs& t, cudaS
   return HBL_OK;
 }
 
-// Token counts up to this bound run on CUDA cores when the codes come packed two per byte.
+// Token counts up to this bound run on CUDA cores (weight bytes bound the product there).
 constexpr int kDecodeMaxM = 8;
 // From this token count on, the product runs on SM pairs (256 x 256 tiles).
 constexpr int kPairMinM = 256;
@@ -375,7 +413,7 @@ hbl_status run_gemm(const void* codes, int fmt, int abits, const float* s_x, con
   const BlobLayout bl = blob_layout(K, N);
   const uint8_t* blob = static_cast<const uint8_t*>(packed);
   const bool packed4 = (abits == 4 && fmt == HBL_CODES_PACKED);
-  if (packed4 && M <= kDecodeMaxM) {
+  if (M <= kDecodeMaxM) {
     DecodeArgs d;
     d.m0 = 0;
     d.codes = static_cast<const uint8_t*>(codes);

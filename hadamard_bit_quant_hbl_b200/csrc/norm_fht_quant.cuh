@@ -42,6 +42,7 @@ struct NfqArgs {
   int slots;          // blocks of a row transformed concurrently (threads per row = slots * P)
   int rows;           // token rows per group
   int groups;         // ceil(M / rows)
+  int pf_dist;        // a CTA prefetches the rows of group blockIdx.x + pf_dist into L2 (0 = none)
 };
 
 // ---------------------------------------------------------------- compile-time plan
@@ -137,14 +138,17 @@ struct SwzBases {
 
 // Butterfly stages on register-index bits 0 .. NSTAGE-1 of v (E values stored as E/2 float2;
 // register r lives in v[r >> 1].x/.y). Sylvester order: (a, b) at (j, j+h) becomes (a+b, a-b).
-template <int E, int NSTAGE>
+// With SKIP0 the stage on register bit 0 has already been applied by the caller.
+template <int E, int NSTAGE, bool SKIP0 = false>
 __device__ __forceinline__ void fwht_regs2(float2 (&v)[E / 2]) {
   // register bit 0: the two halves of each float2
+  if constexpr (!SKIP0) {
 #pragma unroll
-  for (int j = 0; j < E / 2; ++j) {
-    const float a = v[j].x, b = v[j].y;
-    v[j].x = a + b;
-    v[j].y = a - b;
+    for (int j = 0; j < E / 2; ++j) {
+      const float a = v[j].x, b = v[j].y;
+      v[j].x = a + b;
+      v[j].y = a - b;
+    }
   }
   const float2 neg1 = make_float2(-1.f, -1.f);
 #pragma unroll
@@ -164,9 +168,11 @@ __device__ __forceinline__ void fwht_regs2(float2 (&v)[E / 2]) {
 
 // Largest CTA a plan is launched with, and the register cap that lets several such CTAs share
 // an SM (the big transforms hold 128 values per thread).
+// (The block-256 plan runs 352-thread CTAs of 32 values per thread: two of them share an SM
+// only at <= 72 registers, since each SM quarter holds 16384 registers and gets 6 of the 22 warps.)
 constexpr int nfq_max_threads(int L) { return L >= 11 ? 256 : 512; }
 constexpr int nfq_max_regs(int EB, int R) {
-  return ((1 << EB) * R) >= 128 ? 168 : (((1 << EB) * R) >= 64 ? 128 : 96);
+  return ((1 << EB) * R) >= 128 ? 168 : (((1 << EB) * R) >= 64 ? 128 : (((1 << EB) * R) >= 32 ? 72 : 64));
 }
 
 // 16-byte streaming load that bypasses L1 (every input byte is read once).
@@ -176,6 +182,18 @@ __device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
+}
+
+// First butterfly stage straight from a word holding two bf16 features a (low half) and b (high
+// half): (a + b, a - b) in fp32, with a read as bf16 by the add itself (exact widening).
+__device__ __forceinline__ float2 bf16x2_butterfly(uint32_t u) {
+  const float b = __uint_as_float(u & 0xffff0000u);
+  float2 r;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.bf16 %0, lo, %3;\n\tsub.rn.f32.bf16 %1, lo, %3;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "r"(u), "f"(b));
+  return r;
 }
 
 // QM: 0 = a8 absmax, 1 = a4 absmean, 2 = a4 absmax
@@ -203,52 +221,67 @@ __global__ void __maxnreg__(nfq_max_regs(EB, R)) norm_fht_quant_kernel(const Nfq
   const int g = blockIdx.x;
   const int row = g * rows + rloc;
   const bool live_row = row < a.M;
+  // Rows past M (last group only) and padding blocks past nb compute on live data and store
+  // nothing, so that every load is unconditional.
+  const int srow = live_row ? row : a.M - 1;
+
+  // a later group's rows into L2 while this group loads and computes
+  if (tid == 0 && a.pf_dist > 0 && g + a.pf_dist < a.groups) {
+    const int g2 = g + a.pf_dist;
+    const uint32_t bytes = (uint32_t)min(rows, a.M - g2 * rows) * (uint32_t)K * 2u;
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.X + (size_t)g2 * rows * K), "r"(bytes)
+                 : "memory");
+  }
 
   constexpr float kQ = QM == 0 ? 127.f : (QM == 1 ? 2.6457513110645906f : 7.f);
   constexpr int kLo = QM == 0 ? -128 : -8, kHi = QM == 0 ? 127 : 7;
   constexpr bool kAbsmax = QM != 1;
 
   // ---- 1. layout 1 straight from global memory (16-byte vectors, every load issued before the
-  // first use), sum of squares (+ gain)
+  // first use), sum of squares; without a gain the first butterfly stage (index bit 0, the two
+  // halves of a bf16 pair) is taken while widening.
   float2 v[R][E / 2];
-  float2 ss2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float ss = 0.f;
   {
     uint4 w[R][NV];
 #pragma unroll
     for (int rho = 0; rho < R; ++rho) {
       const int blk = slot + rho * a.slots;
-      const bool live = live_row && blk < nb;
-      const uint16_t* src = a.X + (size_t)row * K + (size_t)blk * n + (pt << 3);
+      const uint16_t* src = a.X + (size_t)srow * K + (size_t)(blk < nb ? blk : 0) * n + (pt << 3);
 #pragma unroll
-      for (int vv = 0; vv < NV; ++vv) w[rho][vv] = live ? ldg_stream_v4(src + (vv << Pl::TOP)) : make_uint4(0u, 0u, 0u, 0u);
+      for (int vv = 0; vv < NV; ++vv) w[rho][vv] = ldg_stream_v4(src + (vv << Pl::TOP));
     }
 #pragma unroll
     for (int rho = 0; rho < R; ++rho) {
       const int blk = slot + rho * a.slots;
+      float2 ss2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int vv = 0; vv < NV; ++vv) {
         const uint32_t u[4] = {w[rho][vv].x, w[rho][vv].y, w[rho][vv].z, w[rho][vv].w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          // bf16 -> fp32 on the integer/logic units: low half moved up by a byte permute
-          float2 f = make_float2(__uint_as_float(__byte_perm(u[i], 0u, 0x1044)), __uint_as_float(u[i] & 0xffff0000u));
-          ss2[i] = __ffma2_rn(f, f, ss2[i]);  // independent chains
+          float2 f;
           if constexpr (HAS_GAIN) {
-            if (live_row && blk < nb) {
-              const float2 gg = *reinterpret_cast<const float2*>(a.gain + (size_t)blk * n + (vv << Pl::TOP) +
-                                                                 (pt << 3) + 2 * i);
-              f = __fmul2_rn(f, gg);
-            }
+            f = make_float2(__uint_as_float(u[i] << 16), __uint_as_float(u[i] & 0xffff0000u));
+            ss2[i] = __ffma2_rn(f, f, ss2[i]);
+            const float2 gg = *reinterpret_cast<const float2*>(a.gain + (size_t)(blk < nb ? blk : 0) * n +
+                                                               (vv << Pl::TOP) + (pt << 3) + 2 * i);
+            f = __fmul2_rn(f, gg);
+          } else {
+            f = bf16x2_butterfly(u[i]);
+            ss2[i] = __ffma2_rn(f, f, ss2[i]);  // (a+b)^2 + (a-b)^2 = 2 (a^2 + b^2)
           }
           v[rho][vv * 4 + i] = f;
         }
       }
+      const float ssr = ((ss2[0].x + ss2[0].y) + (ss2[1].x + ss2[1].y)) + ((ss2[2].x + ss2[2].y) + (ss2[3].x + ss2[3].y));
+      if (blk < nb) ss += ssr;
     }
   }
-  float ss = ((ss2[0].x + ss2[0].y) + (ss2[1].x + ss2[1].y)) + ((ss2[2].x + ss2[2].y) + (ss2[3].x + ss2[3].y));
+  if constexpr (!HAS_GAIN) ss *= 0.5f;
 
 #pragma unroll
-  for (int rho = 0; rho < R; ++rho) fwht_regs2<E, EB>(v[rho]);
+  for (int rho = 0; rho < R; ++rho) fwht_regs2<E, EB, !HAS_GAIN>(v[rho]);
 
   // ---- 2. regroup through shared memory (index within the CTA buffer: (rloc*nb + blk)*n + i)
   const uint32_t rowbase = (uint32_t)rloc * (uint32_t)K;
@@ -268,44 +301,37 @@ __global__ void __maxnreg__(nfq_max_regs(EB, R)) norm_fht_quant_kernel(const Nfq
 #pragma unroll
   for (int rho = 0; rho < R; ++rho) {
     const int blk = slot + rho * a.slots;
-    if (blk < nb) {
-      const SwzBases<Pl> sb(rowbase + ((uint32_t)blk << L) + (uint32_t)Pl::idx2(pt, 0));
+    const SwzBases<Pl> sb(rowbase + ((uint32_t)(blk < nb ? blk : 0) << L) + (uint32_t)Pl::idx2(pt, 0));
 #pragma unroll
-      for (int r = 0; r < E; r += 2) {
-        v[rho][r / 2].x = fbuf[sb.at((uint32_t)Pl::idx2(0, r))];
-        v[rho][r / 2].y = fbuf[sb.at((uint32_t)Pl::idx2(0, r + 1))];
-      }
-      fwht_regs2<E, S2>(v[rho]);
-    } else {
-#pragma unroll
-      for (int r = 0; r < E / 2; ++r) v[rho][r] = make_float2(0.f, 0.f);
+    for (int r = 0; r < E; r += 2) {
+      v[rho][r / 2].x = fbuf[sb.at((uint32_t)Pl::idx2(0, r))];
+      v[rho][r / 2].y = fbuf[sb.at((uint32_t)Pl::idx2(0, r + 1))];
     }
+    fwht_regs2<E, S2>(v[rho]);
   }
 
   // ---- 3. row statistics: sum |y| as pairwise sums folded into fp32x2 chains, or max |y|
-  float st;
-  if constexpr (kAbsmax) {
-    float sta[4] = {0.f, 0.f, 0.f, 0.f};
+  float st = 0.f;
 #pragma unroll
-    for (int rho = 0; rho < R; ++rho)
+  for (int rho = 0; rho < R; ++rho) {
+    const int blk = slot + rho * a.slots;
+    float str;
+    if constexpr (kAbsmax) {
+      float sta[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int r = 0; r < E / 2; ++r) {
-        float& acc = sta[(rho * (E / 2) + r) & 3];
-        acc = fmaxf(acc, fmaxf(fabsf(v[rho][r].x), fabsf(v[rho][r].y)));
-      }
-    st = fmaxf(fmaxf(sta[0], sta[1]), fmaxf(sta[2], sta[3]));
-  } else {
-    float2 sta2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-    for (int rho = 0; rho < R; ++rho)
+      for (int r = 0; r < E / 2; ++r) sta[r & 3] = fmaxf(sta[r & 3], fmaxf(fabsf(v[rho][r].x), fabsf(v[rho][r].y)));
+      str = fmaxf(fmaxf(sta[0], sta[1]), fmaxf(sta[2], sta[3]));
+    } else {
+      float2 sta2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int r = 0; r < E / 2; r += 2) {
         const float2 t = make_float2(fabsf(v[rho][r].x) + fabsf(v[rho][r].y),
                                      fabsf(v[rho][r + 1].x) + fabsf(v[rho][r + 1].y));
-        float2& acc = sta2[(rho * (E / 4) + r / 2) & 3];
-        acc = __fadd2_rn(acc, t);
+        sta2[(r / 2) & 3] = __fadd2_rn(sta2[(r / 2) & 3], t);
       }
-    st = ((sta2[0].x + sta2[0].y) + (sta2[1].x + sta2[1].y)) + ((sta2[2].x + sta2[2].y) + (sta2[3].x + sta2[3].y));
+      str = ((sta2[0].x + sta2[0].y) + (sta2[1].x + sta2[1].y)) + ((sta2[2].x + sta2[2].y) + (sta2[3].x + sta2[3].y));
+    }
+    if (blk < nb) st = kAbsmax ? fmaxf(st, str) : st + str;
   }
   if (tpr >= 32) {
 #pragma unroll
@@ -394,18 +420,20 @@ __global__ void __maxnreg__(nfq_max_regs(EB, R)) norm_fht_quant_kernel(const Nfq
   }
   __syncthreads();
 
-  // ---- 6. stream codes out in natural order, 32 consecutive codes per unit
-  const int upr = K / 32;  // units per row
+  // ---- 6. stream codes out in natural order, 32 consecutive codes per unit. A thread owns at
+  // most R*E/32 units (units tid, tid + blockDim, ...). With nb == 1 a row has 2^(L-5) units;
+  // with nb > 1 the CTA holds one row.
+  const int upr = K / 32;
+  const int units = rows * upr;
   const bool packed4 = (a.fmt == 0) && (QM != 0);
-  // thread tid handles units tid, tid + blockDim, ... of the CTA's rows * upr units; walk them
-  // row by row without dividing
-  int rl = 0, vcol = tid;
-  while (vcol >= upr && rl < rows) { vcol -= upr; ++rl; }
-  for (; rl < rows; vcol += blockDim.x) {
-    while (vcol >= upr) { vcol -= upr; ++rl; }
-    if (rl >= rows) break;
+#pragma unroll
+  for (int it = 0; it < (R * E + 31) / 32; ++it) {
+    const int unit = tid + it * (int)blockDim.x;
+    if (unit >= units) break;
+    const int rl = nb == 1 ? (unit >> (L - 5)) : 0;
+    const int vcol = unit - rl * upr;
     const int grow = g * rows + rl;
-    if (grow >= a.M) break;  // rows past M are the CTA's last ones
+    if (grow >= a.M) break;  // later units belong to later rows
     const uint8_t* srcc = cbuf + (size_t)rl * 8 * crow + 4 * vcol;
     uint32_t w[8];
 #pragma unroll

@@ -185,14 +185,20 @@ def run_gemm_with_oracle_codes(q, t, s, alpha, fmt, abits):
 
 
 GEMM_CASES = [
-    # (M, K, N, abits, fmt)  -- M <= 8 runs on CUDA cores, larger M on tcgen05
+    # (M, K, N, abits, fmt)  -- M <= 8 runs on CUDA cores, up to 256 on swapped tcgen05 tiles,
+    # larger M on SM pairs
     (1, 256, 8, 4, hbl.HBL_CODES_PACKED),
     (1, 16384, 264, 4, hbl.HBL_CODES_PACKED),
     (2, 4096, 128, 8, hbl.HBL_CODES_PACKED),
     (3, 11008, 72, 4, hbl.HBL_CODES_I8),
     (5, 2048, 520, 4, hbl.HBL_CODES_PACKED),
     (8, 32768, 24, 4, hbl.HBL_CODES_PACKED),
+    (1, 4096, 4096, 4, hbl.HBL_CODES_I8),
+    (7, 16384, 136, 4, hbl.HBL_CODES_I8),
     (9, 256, 8, 4, hbl.HBL_CODES_I8),
+    (16, 4096, 264, 4, hbl.HBL_CODES_I8),
+    (64, 16384, 128, 4, hbl.HBL_CODES_I8),
+    (255, 2048, 136, 8, hbl.HBL_CODES_I8),
     (128, 1024, 256, 8, hbl.HBL_CODES_I8),
     (300, 2048, 520, 4, hbl.HBL_CODES_I8),
     (257, 11008, 264, 4, hbl.HBL_CODES_I8),
