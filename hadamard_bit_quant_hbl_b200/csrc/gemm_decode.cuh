@@ -9,14 +9,20 @@
 // is 4 KB of contiguous memory) and every byte is read once, with coalesced 16-byte loads.
 //
 // A cluster of S CTAs shares one 128-feature tile and splits K: CTA r owns a contiguous run of
-// k-blocks. Within a k-block, thread t owns feature t/2 and half t%2 of the block (64 k, one
-// 16-byte load; the 256 threads read the 4 KB tile in order). Two chunks of k-blocks are in
-// flight per thread (double buffering in registers), the first two issued before anything else.
-// A 2-bit group is widened with a shift and a mask into four unsigned bytes c that feed __dp4a
-// against int8 activations staged in shared memory:  sum_k q t = sum_k q c - sum_k q.
-// The two halves of a feature meet in a warp shuffle; the cluster's partial sums meet in
-// distributed shared memory (fixed order), so results are exact and reproducible and no global
-// workspace is needed.
+// k-blocks, which the TMA engine streams into a ring of shared-memory stages (16 KB bulk copies,
+// completion on mbarriers, every wait bounded); per-thread global loads could not keep enough
+// bytes in flight. Within a k-block, thread t owns feature t/2 and half t%2 of the block (64 k,
+// one conflict-free 16-byte shared load). A word holds 16 codes, c of k = 16w + 4s + b at bits
+// 8b + 2s; masking plane s in place leaves bytes c * 4^s, which feed __dp4a (unsigned x signed)
+// against the int8 activations of k-group s staged in shared memory, one accumulator per plane;
+// the planes recombine exactly as acc0 + acc1 / 4 + acc2 / 16 + acc3 / 64, and
+//   sum_k q t = sum_k q c - sum_k q.
+// The kernel may start while the activation kernel before it still runs (programmatic
+// dependent launch): it issues its weight copies first and waits for that kernel only before
+// it reads the codes. The two halves of a feature meet in a warp shuffle; each CTA
+// then stores its partial sums straight into the shared memory of the CTA that owns the feature
+// (one slot per peer), so that one cluster barrier suffices and each owner sums its slots in a
+// fixed order: results are exact and reproducible, and no global workspace is needed.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -26,10 +32,6 @@
 namespace hbl {
 
 constexpr int kDecThreads = 256;
-
-// k-blocks per chunk of weight loads (two chunks in flight); fewer when many token rows hold
-// registers
-constexpr int dec_unroll(int MT) { return MT >= 8 ? 4 : 8; }
 
 struct DecodeArgs {
   const uint8_t* codes;  // activation codes: int8 [M][K] or packed int4 [M][K/2]
@@ -56,21 +58,28 @@ __device__ __forceinline__ void widen_int4x8(uint32_t x, uint32_t& lo, uint32_t&
   hi = __byte_perm(ev, od, 0x7362);
 }
 
-__device__ __forceinline__ uint4 ldg_stream_u4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
+// Dot product of four unsigned bytes of a with four signed bytes of b, plus c.
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
 }
 
-// Shared memory: the partial sums [MT][128] int32 (first, at the same offset in every CTA of the
-// cluster: peers read them there), then int8 activations [MT][range] (range = this CTA's k count).
+// Shared memory: the peers' partial sums [S][MT][FO] int32 for the FO features this CTA owns
+// (first, at the same offset in every CTA of the cluster: peers write them there), then the
+// weight ring [kDecStages][kDecChunk * 4 KB], then int8 activations [MT][range] (range = this
+// CTA's k count). CTA r owns features [r * FO, (r + 1) * FO) of the tile, FO = ceil(128 / S).
+__host__ __device__ constexpr int dec_slot_bytes(int S, int MT) { return (int)round_up((size_t)S * MT * ((128 + S - 1) / S) * 4, 16); }
+constexpr int kDecChunk = 4;   // k-blocks per bulk copy (16 KB)
+constexpr int kDecStages = 4;  // copies in flight
+constexpr int kDecRingBytes = kDecStages * kDecChunk * 4096;
+
 template <int MT>
 __global__ void __launch_bounds__(kDecThreads, 2) gemm_decode_kernel(const DecodeArgs a) {
-  constexpr int U = dec_unroll(MT);
-  extern __shared__ __align__(16) uint8_t dec_smem[];
+  extern __shared__ __align__(128) uint8_t dec_smem[];
   __shared__ int32_t qred[MT][kDecThreads / 32];
+  __shared__ __align__(8) uint64_t full[kDecStages];
+  __shared__ volatile int abort_flag;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S = a.S;
@@ -80,24 +89,33 @@ __global__ void __launch_bounds__(kDecThreads, 2) gemm_decode_kernel(const Decod
   const int KB = a.K >> 7;
   const int kb0 = (int)(((long)KB * rank) / S), kb1 = (int)(((long)KB * (rank + 1)) / S);
   const int nkb = kb1 - kb0;
+  const int nch = (nkb + kDecChunk - 1) / kDecChunk;
   const int range = nkb * 128;
-  int32_t* part = reinterpret_cast<int32_t*>(dec_smem);
-  int8_t* act = reinterpret_cast<int8_t*>(dec_smem + MT * 128 * 4);
+  const int FO = (128 + S - 1) / S;
+  int32_t* slots = reinterpret_cast<int32_t*>(dec_smem);
+  uint8_t* ring = dec_smem + dec_slot_bytes(S, MT);
+  int8_t* act = reinterpret_cast<int8_t*>(ring + kDecRingBytes);
+  cluster_arrive_relaxed();  // "this CTA runs"; waited for before the first remote store
 
-  // ---- thread = (feature f, half h) of each k-block. Weight loads go out first (they need
-  // nothing else), two chunks of U k-blocks in flight while the activations are staged.
-  const int f = tid >> 1, h = tid & 1;
-  const uint32_t* wt = a.w2 + ((size_t)tile * KB + kb0) * 1024 + f * 8 + 4 * h;
-  auto load_chunk = [&](uint4 (&w)[U], int i0) {
-#pragma unroll
-    for (int u = 0; u < U; ++u)
-      w[u] = (i0 + u < nkb) ? ldg_stream_u4(wt + (size_t)(i0 + u) * 1024) : make_uint4(0u, 0u, 0u, 0u);
+  // ---- 1. the first kDecStages chunks of this CTA's weight tiles (consecutive in memory)
+  const uint8_t* wsrc = reinterpret_cast<const uint8_t*>(a.w2) + ((size_t)tile * KB + kb0) * 4096;
+  auto issue = [&](int c) {  // one thread
+    const int stg = c % kDecStages;
+    const uint32_t bytes = (uint32_t)min(kDecChunk, nkb - c * kDecChunk) * 4096u;
+    mbar_arrive_expect_tx(&full[stg], bytes);
+    bulk_load_1d(ring + stg * (kDecChunk * 4096), wsrc + (size_t)c * kDecChunk * 4096, bytes, &full[stg]);
   };
-  uint4 wa[U], wb[U];
-  load_chunk(wa, 0);
-  load_chunk(wb, U);
+  int issued = 0;  // chunks handed to the TMA engine (thread 0)
+  if (tid == 0) {
+    abort_flag = 0;
+    for (int i = 0; i < kDecStages; ++i) mbar_init(&full[i], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (; issued < nch && issued < kDecStages; ++issued) issue(issued);
+  }
 
-  // ---- stage this CTA's activations (16 codes per step) and their per-token sums
+  // ---- 2. stage the activations and their per-token sums (packed rows widened). Until here
+  // the kernel touched only its weights; the codes may come from the kernel before it
+  pdl_wait();
   int qs[MT];
 #pragma unroll
   for (int m = 0; m < MT; ++m) qs[m] = 0;
@@ -132,45 +150,71 @@ __global__ void __launch_bounds__(kDecThreads, 2) gemm_decode_kernel(const Decod
     for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (lane == 0) qred[m][warp] = v;
   }
-  __syncthreads();
+  __syncthreads();  // barriers initialised, activations staged
 
-  // ---- widen and multiply, one chunk while the next one's loads are in flight
+  // ---- 3. per chunk: wait (bounded; the outcome is voted so that all threads leave together),
+  // refill the stage the previous chunk used (every thread is past it), widen and multiply;
+  // thread = (feature f, half h) reads the 16 bytes at f * 32 + h * 16 of each 4 KB tile
+  const int f = tid >> 1, h = tid & 1;
   const int8_t* ab = act + 64 * h;
-  int acc[MT];
+  int accp[4][MT];  // per bit plane
 #pragma unroll
-  for (int m = 0; m < MT; ++m) acc[m] = 0;
-  auto compute_chunk = [&](const uint4 (&w)[U], int i0) {
+  for (int p = 0; p < 4; ++p)
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      if (i0 + u < nkb) {
-        const uint32_t ww[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
-        const int8_t* ak = ab + (i0 + u) * 128;
+    for (int m = 0; m < MT; ++m) accp[p][m] = 0;
+  // one k-block: 4 words of 16 codes, each plane against its activation word
+  auto kblock = [&](const uint8_t* wp, const int8_t* ak) {
+    const uint4 wv = *reinterpret_cast<const uint4*>(wp);
+    const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {  // word i: 16 features k = 64h + 16i + 4s + b
-          uint4 q[MT];
+    for (int i = 0; i < 4; ++i) {  // word i: codes of k = 64h + 16i + 4s + b
+      uint4 q[MT];
 #pragma unroll
-          for (int m = 0; m < MT; ++m) q[m] = *reinterpret_cast<const uint4*>(ak + (size_t)m * range + 16 * i);
+      for (int m = 0; m < MT; ++m) q[m] = *reinterpret_cast<const uint4*>(ak + (size_t)m * range + 16 * i);
 #pragma unroll
-          for (int s = 0; s < 4; ++s) {
-            const int cw = (int)((ww[i] >> (2 * s)) & 0x03030303u);
+      for (int p = 0; p < 4; ++p) {
+        const uint32_t cw = ww[i] & (0x03030303u << (2 * p));  // bytes c * 4^p
 #pragma unroll
-            for (int m = 0; m < MT; ++m) {
-              const uint32_t qw = s == 0 ? q[m].x : s == 1 ? q[m].y : s == 2 ? q[m].z : q[m].w;
-              acc[m] = __dp4a((int)qw, cw, acc[m]);
-            }
-          }
+        for (int m = 0; m < MT; ++m) {
+          const uint32_t qw = p == 0 ? q[m].x : p == 1 ? q[m].y : p == 2 ? q[m].z : q[m].w;
+          accp[p][m] = dp4a_us(cw, qw, accp[p][m]);
         }
       }
     }
   };
-  for (int i0 = 0; i0 < nkb; i0 += 2 * U) {
-    compute_chunk(wa, i0);
-    if (i0 + 2 * U < nkb) load_chunk(wa, i0 + 2 * U);
-    if (i0 + U < nkb) compute_chunk(wb, i0 + U);
-    if (i0 + 3 * U < nkb) load_chunk(wb, i0 + 3 * U);
+  int c = 0;
+  for (; c < nch; ++c) {
+    const int stg = c % kDecStages;
+    const bool ok = mbar_wait(&full[stg], (uint32_t)(c / kDecStages) & 1u, &abort_flag);
+    if (!__syncthreads_and(ok)) break;
+    if (tid == 0 && c >= 1 && issued < nch) issue(issued++);  // chunk c + 3 into chunk c - 1's stage
+    const uint8_t* wbase = ring + stg * (kDecChunk * 4096) + f * 32 + h * 16;
+    const int8_t* abase = ab + c * (kDecChunk * 128);
+    if ((c + 1) * kDecChunk <= nkb) {
+#pragma unroll
+      for (int u = 0; u < kDecChunk; ++u) kblock(wbase + u * 4096, abase + u * 128);
+    } else {
+      for (int u = 0; c * kDecChunk + u < nkb; ++u) kblock(wbase + u * 4096, abase + u * 128);
+    }
+  }
+  int acc[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m)  // each plane's sum is a multiple of 4^p: exact
+    acc[m] = accp[0][m] + (accp[1][m] >> 2) + (accp[2][m] >> 4) + (accp[3][m] >> 6);
+  // an aborted wait leaves no copy in flight into shared memory when the CTA exits
+  if (tid == 0 && c < nch) {
+    for (int d = c; d < issued; ++d) {
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(&full[d % kDecStages], (uint32_t)(d / kDecStages) & 1u) &&
+             globaltimer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
   }
 
-  // ---- the two halves of a feature, minus this CTA's sum of q, into shared memory
+  // ---- 4. the two halves of a feature, minus this CTA's sum of q, into the owner's slot
+  const int owner = f / FO, fo = f - owner * FO;
+  const uint32_t slot0 = smem_u32(slots);
+  cluster_wait();  // every CTA of the cluster is running
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
     acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], 1);
@@ -178,30 +222,25 @@ __global__ void __launch_bounds__(kDecThreads, 2) gemm_decode_kernel(const Decod
       int qsum = 0;
 #pragma unroll
       for (int w = 0; w < kDecThreads / 32; ++w) qsum += qred[m][w];
-      part[m * 128 + f] = acc[m] - qsum;
+      const uint32_t off = (uint32_t)((((int)rank * MT + m) * FO + fo) * 4);
+      st_shared_cluster_u32(mapa_shared(slot0 + off, (uint32_t)owner), (uint32_t)(acc[m] - qsum));
     }
   }
-  cluster_sync_all();
+  cluster_sync_all();  // every peer's slots have landed; after this each CTA reads only its own
 
-  // ---- reduce across the cluster (fixed order), dequant, store
-  const uint32_t part0 = smem_u32(part);
-  for (int e = (int)rank * kDecThreads + tid; e < MT * 128; e += S * kDecThreads) {
-    const int m = e >> 7, fl = e & 127;
-    const int n = n0 + fl, row = a.m0 + m;
-    if (row >= a.M || n >= a.N) continue;
-    uint32_t pv[8];
-#pragma unroll
-    for (int p = 0; p < 8; ++p)  // all remote loads in flight before the sum
-      pv[p] = p < S ? ld_shared_cluster_u32(mapa_shared(part0 + (uint32_t)e * 4u, (uint32_t)p)) : 0u;
+  // ---- 5. sum the slots of the owned features (fixed order), dequant, store
+  for (int e = tid; e < MT * FO; e += kDecThreads) {
+    const int m = e / FO, fl = e - m * FO;
+    const int ft = (int)rank * FO + fl;
+    const int n = n0 + ft, row = a.m0 + m;
+    if (ft >= 128 || row >= a.M || n >= a.N) continue;
     int32_t accv = 0;
-#pragma unroll
-    for (int p = 0; p < 8; ++p) accv += (int32_t)pv[p];
+    for (int p = 0; p < S; ++p) accv += slots[(p * MT + m) * FO + fl];
     const float y = (float)accv * (a.s_x[row] * a.alpha);
     if (a.out_bf16) reinterpret_cast<__nv_bfloat16*>(a.Y)[(size_t)row * a.N + n] = __float2bfloat16_rn(y);
     else reinterpret_cast<float*>(a.Y)[(size_t)row * a.N + n] = y;
     if (a.acc_debug) a.acc_debug[(size_t)row * a.N + n] = accv;
   }
-  cluster_sync_all();  // no CTA leaves while a peer may still read its shared memory
 }
 
 }  // namespace hbl

@@ -210,13 +210,15 @@ hbl_status launch_decode_t(const DecodeArgs& a, int smem, cudaStream_t s) {
   cfg.blockDim = dim3(kDecThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = a.S;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may overlap the kernel before
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, gemm_decode_kernel<MT>, a);
   if (e != cudaSuccess) return cuda_fail(e);
   HBL_CHECK_LAUNCH();
@@ -225,7 +227,7 @@ hbl_status launch_decode_t(const DecodeArgs& a, int smem, cudaStream_t s) {
 
 // One launch per slice of up to 8 token rows. A cluster of S CTAs splits K for each 128-feature
 // tile: S is chosen so that about two CTAs run per SM, and large enough that the CTA's staged
-// activations stay within 64 KB.
+// activations stay within 32 KB (next to the 64 KB weight ring).
 hbl_status run_decode(const DecodeArgs& a0, cudaStream_t s) {
   DecodeArgs a = a0;
   int dev = 0;
@@ -236,14 +238,14 @@ hbl_status run_decode(const DecodeArgs& a0, cudaStream_t s) {
     const int left = a0.M - a.m0;
     const int MT = left == 1 ? 1 : left == 2 ? 2 : left <= 4 ? 4 : 8;
     int S = (2 * device_sms(dev) + ntiles - 1) / ntiles;
-    const int smin = (a.K * MT + 65535) / 65536;
+    const int smin = (a.K * MT + 32767) / 32768;
     if (S < smin) S = smin;
     if (S > 8) S = 8;
     if (S > KB) S = KB;
     if (S < 1) S = 1;
     a.S = S;
     const int range = (KB + S - 1) / S * 128;
-    const int smem = MT * range + MT * 128 * 4;
+    const int smem = dec_slot_bytes(S, MT) + kDecRingBytes + MT * range;
     hbl_status st;
     switch (MT) {
       case 1: st = launch_decode_t<1>(a, smem, s); break;

@@ -225,6 +225,10 @@ __global__ void __maxnreg__(nfq_max_regs(EB, R)) norm_fht_quant_kernel(const Nfq
   // nothing, so that every load is unconditional.
   const int srow = live_row ? row : a.M - 1;
 
+  // the product that consumes these codes may start now: it streams its weights, which this
+  // kernel does not write, and waits for this kernel's completion before it reads the codes
+  pdl_launch_dependents();
+
   // a later group's rows into L2 while this group loads and computes
   if (tid == 0 && a.pf_dist > 0 && g + a.pf_dist < a.groups) {
     const int g2 = g + a.pf_dist;
