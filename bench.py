@@ -41,7 +41,7 @@ WORKLOAD = ("7B-like H-BitLinear layer pair: Wo 4096->4096 + Wdown 16384->4096, 
 # source it was taken on (reported as null once the source has changed).
 NCU_TRAFFIC = {
     # profiles/gemm_tc2_wdown_7b_m8192.md: dram__bytes_read.sum + dram__bytes_write.sum
-    "gemm_tc2[wdown_7b_a4]": {"bytes": 607.685376e6 + 73.879552e6, "src": "gemm_tc2.cuh", "sha": "179b5ae7b9be7658"},
+    "gemm_tc2[wdown_7b_a4]": {"bytes": 611.340544e6 + 73.249024e6, "src": "gemm_tc2.cuh", "sha": "8eab555aa3d677d4"},
 }
 
 
@@ -49,7 +49,13 @@ def product_kernel(M):
     """Name and source file of the product kernel hbl_ternary_gemm runs for M tokens."""
     if M <= 8:
         return "gemm_decode", "gemm_decode.cuh"
-    return ("gemm_tc2", "gemm_tc2.cuh") if M >= 256 else ("gemm_tc", "gemm_tc.cuh")
+    return ("gemm_swap", "gemm_swap.cuh") if M <= 256 else ("gemm_tc2", "gemm_tc2.cuh")
+
+
+def weight_bytes(M, K, N):
+    """Weight bytes the product kernel reads for M tokens: the 2-bit section up to 256 tokens,
+    the int8 section above."""
+    return (K * N) // 4 if M <= 256 else K * N
 
 
 def peaks():
@@ -296,7 +302,7 @@ def run_ours(args, world, rank, local):
     h2d = sum(L["X"].numel() * 2 for L in layers)
     d2h = sum(L["Y"].numel() * 2 for L in layers)
 
-    # ---- token-count sweep of the same layer pair (CUDA-graph replay, L2 flushed before each step)
+    # ---- token-count sweep of the same layer pair (CUDA-graph replay over rotating weight copies)
     sweep = [] if args.no_sweep else run_sweep(layers, dev, args)
 
     st = hbl.hbl_device_status()
@@ -361,15 +367,17 @@ def run_ours(args, world, rank, local):
 
 
 def run_sweep(layers, dev, args):
-    """Per token count M: one step = hbl_forward of Wo then Wdown on the first M rows, captured
-    in a CUDA graph; before every timed replay a 256 MB buffer is written so that weights and
-    activations come from HBM, not L2. Reports tokens/s, effective TOPS and the bandwidth on the
-    2-bit (M <= 8) or int8 weight bytes the product reads."""
+    """Per token count M: one step = hbl_forward of Wo then Wdown on the first M rows. A CUDA
+    graph holds R consecutive steps, each on its own copy of the packed weights, so that the
+    weight bytes of a step come from HBM (R copies of the bytes the product reads exceed L2)
+    without a flush kernel in the timed region. Reports tokens/s, effective TOPS and the
+    bandwidth on the weight bytes the product reads (2-bit up to 256 tokens, int8 above)."""
     import torch
 
     import hadamard_bit_quant_hbl_b200 as hbl
 
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    R = 8
+    copies = [[L["packed"]] + [L["packed"].clone() for _ in range(R - 1)] for L in layers]
     out = []
     for M in SWEEP_TOKENS:
         bufs = []
@@ -379,41 +387,62 @@ def run_sweep(layers, dev, args):
             ws = torch.empty(hbl.hbl_forward_workspace(M, sp.K, hbl.HBL_Q_A4_ABSMEAN), dtype=torch.uint8, device=dev)
             bufs.append((L, L["X"][:M], Y, ws))
 
-        def step(s):
-            for L, X, Y, ws in bufs:
-                hbl.hbl_forward(X, L["packed"], L["alpha"], L["spec"].N, None, L["spec"].had_block,
-                                hbl.HBL_Q_A4_ABSMEAN, workspace=ws, Y=Y, out_dtype=hbl.HBL_OUT_BF16, stream=s)
+        def steps(s):
+            for r in range(R):
+                for i, (L, X, Y, ws) in enumerate(bufs):
+                    hbl.hbl_forward(X, copies[i][r], L["alpha"], L["spec"].N, None, L["spec"].had_block,
+                                    hbl.HBL_Q_A4_ABSMEAN, workspace=ws, Y=Y, out_dtype=hbl.HBL_OUT_BF16, stream=s)
 
         cap = torch.cuda.Stream(dev)
         with torch.cuda.stream(cap):
-            step(cap.cuda_stream)  # warm-up outside capture (one-time host setup)
+            steps(cap.cuda_stream)  # warm-up outside capture (one-time host setup)
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=cap):
-            step(cap.cuda_stream)
+            steps(cap.cuda_stream)
         torch.cuda.synchronize()
-        reps = max(20, min(args.sweep_steps, 200))
+        reps = max(5, min(args.sweep_steps // R, 50))
         for _ in range(3):
             g.replay()
         torch.cuda.synchronize()
-        tot = 0.0
         cur = torch.cuda.current_stream(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(cur)
         for _ in range(reps):
-            flush.fill_(1)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(cur)
             g.replay()
-            e1.record(cur)
-            e1.synchronize()
-            tot += e0.elapsed_time(e1)
-        ms = tot / reps
-        wbytes = sum((L["spec"].K * L["spec"].N) // (4 if M <= 8 else 1) for L in layers)
+        e1.record(cur)
+        e1.synchronize()
+        ms = e0.elapsed_time(e1) / (reps * R)
+        wbytes = sum(weight_bytes(M, L["spec"].K, L["spec"].N) for L in layers)
         ops = sum(2.0 * M * L["spec"].N * L["spec"].K for L in layers)
         out.append({"M": M, "ms_per_step": ms, "tokens_per_s": M / (ms / 1e3), "effective_tops": ops / (ms / 1e3) / 1e12,
                     "weight_bytes": wbytes, "weight_GBps": wbytes / (ms / 1e3) / 1e9,
-                    "product": "cuda-core 2-bit" if M <= 8 else ("tcgen05 pair" if M >= 256 else "tcgen05")})
+                    "product": product_kernel(M)[0],
+                    "l2": f"{R} weight copies rotated per graph replay"})
         del g
+    del copies
     return out
+
+
+def run_profile_product(M):
+    """Runs the activation kernel once and the product three times on the Wdown shape with M
+    tokens (a small, self-contained target for an ncu capture of one product kernel)."""
+    import torch
+
+    import hadamard_bit_quant_hbl_b200 as hbl
+
+    torch.cuda.set_device(0)
+    spec = inputs.WORKLOADS["wdown_7b_a4"].with_m(M)
+    X = torch.from_numpy(inputs.activations(spec).view(np.int16)).cuda().view(torch.bfloat16)
+    packed, alpha = hbl.hbl_pack_weights(torch.from_numpy(inputs.weights(spec)).cuda())
+    codes, s_x = hbl.hbl_norm_fht_quant(X, None, 0, hbl.HBL_Q_A4_ABSMEAN, 1e-6, 0.0, hbl.HBL_CODES_I8)
+    for _ in range(3):
+        hbl.hbl_ternary_gemm(codes, hbl.HBL_CODES_I8, 4, s_x, packed, alpha, spec.N, spec.K, out_dtype=hbl.HBL_OUT_BF16)
+    torch.cuda.synchronize()
+    st = hbl.hbl_device_status()
+    if st != hbl.HBL_OK:
+        raise RuntimeError(hbl.hbl_status_string(st))
+    print(f"product {product_kernel(M)[0]}: M={M} K={spec.K} N={spec.N}, 3 launches", flush=True)
 
 
 def main():
@@ -428,7 +457,12 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--no-sweep", action="store_true", help="skip the token-count sweep")
     ap.add_argument("--sweep-steps", type=int, default=100)
+    ap.add_argument("--profile-product", type=int, default=0, metavar="M",
+                    help="only run the Wdown product three times with M tokens (an ncu target); no bench line")
     args = ap.parse_args()
+    if args.profile_product:
+        run_profile_product(args.profile_product)
+        return
     world, rank, local = dist_setup(args.gpus) if args.impl == "ours" else (
         int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
     try:

@@ -1,23 +1,13 @@
-// Ternary x low-bit product for prefill-sized token counts on the sm_100a tensor cores.
+// tcgen05 / TMA building blocks shared by the tensor-core product kernels (sm_100a), and the
+// argument block of the product:
 //
 //   Y[m, n] = s_x[m] * alpha * sum_k q[m, k] * t[k, n]
 //
 // The layer's product (BitNet v2 walkthrough article, section "H-BitLinear模塊"). Integer codes
 // (activations in [-8, 7] or [-128, 127], weights in {-1, 0, 1}) are multiplied exactly by
-// tcgen05.mma kind::i8 with int32 accumulation in tensor memory.
-//
-// Structure (one CTA per SM, persistent over 128 x 256 output tiles, 6 warps):
-//   warp 0     TMA producer: 128x128-byte A tile and 256x128-byte B tile per k-block into a
-//              4-stage shared-memory ring (128-byte swizzle), completion on an mbarrier.
-//   warp 1     allocates all 512 TMEM columns (two 256-column accumulators), one thread issues
-//              4 MMAs of K = 32 per k-block and commits to the stage's "empty" barrier and,
-//              after the last k-block, to the accumulator's "full" barrier.
-//   warps 2-5  epilogue: tcgen05.ld 32 lanes x 32 columns at a time, scale by s_x[m] * alpha,
-//              store fp32 or bf16; then release the accumulator so the MMA warp can reuse it
-//              while the next tile's epilogue runs on the other one.
-// Every mbarrier wait is bounded (1 s of wall clock); on time-out the kernel raises the device
-// error flag, stops issuing work, waits (bounded) for its own copies and MMAs, frees TMEM and
-// returns.
+// tcgen05.mma kind::i8 with int32 accumulation in tensor memory: see gemm_tc2.cuh (SM pairs,
+// 256 x 256 tiles, token counts above 256) and gemm_swap.cuh (weights on the MMA's M side, up to
+// 256 tokens).
 #pragma once
 
 #include <cuda.h>
@@ -26,13 +16,6 @@
 #include "common.cuh"
 
 namespace hbl {
-
-constexpr int kTcBM = 128, kTcBN = 256, kTcBK = 128;
-constexpr int kTcStages = 4;
-constexpr int kTcStageA = kTcBM * kTcBK;  // bytes
-constexpr int kTcStageB = kTcBN * kTcBK;
-constexpr int kTcSmem = kTcStages * (kTcStageA + kTcStageB) + 1024;  // + alignment slack
-constexpr int kTcThreads = 192;
 
 struct TcArgs {
   const float* s_x;
@@ -125,194 +108,5 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
 }
 
 // ---------------------------------------------------------------- the kernel
-
-__global__ void __launch_bounds__(kTcThreads, 1)
-gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-               const TcArgs a) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[kTcStages], empty_bar[kTcStages];
-  __shared__ __align__(8) uint64_t accf_bar[2], acce_bar[2], drain_bar;
-  __shared__ uint32_t tmem_base_slot;
-  __shared__ volatile int abort_flag;
-
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* smA = smem;
-  uint8_t* smB = smem + kTcStages * kTcStageA;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int KB = a.K / kTcBK;
-  const int ntiles = a.tiles_m * a.tiles_n;
-
-  if (threadIdx.x == 0) {
-    abort_flag = 0;
-    for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&accf_bar[b], 1);
-      mbar_init(&acce_bar[b], 128);
-    }
-    mbar_init(&drain_bar, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    tma_prefetch_desc(&mapA);
-    tma_prefetch_desc(&mapB);
-  }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;"
-                 ::"r"(smem_u32(&tmem_base_slot)) : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = tmem_base_slot;
-
-  if (warp == 0) {
-    // ---------------- TMA producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int issued[kTcStages] = {0, 0, 0, 0};
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-        const int tm = tile % a.tiles_m, tn = tile / a.tiles_m;
-        for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full_bar[stage], kTcStageA + kTcStageB);
-          tma_load_2d(smA + stage * kTcStageA, &mapA, &full_bar[stage], kb * kTcBK, tm * kTcBM);
-          tma_load_2d(smB + stage * kTcStageB, &mapB, &full_bar[stage], kb * kTcBK, tn * kTcBN);
-          ++issued[stage];
-          if (++stage == kTcStages) { stage = 0; phase ^= 1u; }
-        }
-      }
-      // every copy this thread issued has landed before the CTA may exit
-      for (int s = 0; s < kTcStages; ++s) {
-        if (issued[s] > 0) {
-          // the last phase armed on stage s has parity (issued[s] - 1) & 1
-          if (!mbar_try_wait(&full_bar[s], (uint32_t)((issued[s] - 1) & 1))) {
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(&full_bar[s], (uint32_t)((issued[s] - 1) & 1)) &&
-                   globaltimer_ns() - t0 < kWaitLimitNs) {
-            }
-          }
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(kTcBM, kTcBN);
-      int stage = 0;
-      uint32_t phase = 0;
-      int local = 0;
-      bool ok = true;
-      bool any = false;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++local) {
-        const int buf = local & 1;
-        const uint32_t use = (uint32_t)(local >> 1);  // how many times this buffer was used before
-        if (!mbar_wait(&acce_bar[buf], (use & 1u) ^ 1u, &abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t tmem_d = tmem_base + (uint32_t)(buf * kTcBN);
-        for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&full_bar[stage], phase, &abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(smA + stage * kTcStageA);
-          const uint32_t b_addr = smem_u32(smB + stage * kTcStageB);
-#pragma unroll
-          for (int kk = 0; kk < kTcBK / 32; ++kk) {
-            mma_i8(tmem_d, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32), idesc,
-                   (kb | kk) != 0 ? 1u : 0u);
-          }
-          any = true;
-          mma_commit(&empty_bar[stage]);
-          if (++stage == kTcStages) { stage = 0; phase ^= 1u; }
-        }
-        if (!ok) break;
-        mma_commit(&accf_bar[buf]);
-      }
-      if (!ok && any) {
-        // no MMA may still be running when TMEM is released
-        mma_commit(&drain_bar);
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(&drain_bar, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
-        }
-      }
-    }
-  } else {
-    // ---------------- epilogue: warps 2..5 -> TMEM lane quarter (warp % 4)
-    const int q = warp & 3;
-    int local = 0;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++local) {
-      const int buf = local & 1;
-      const uint32_t use = (uint32_t)(local >> 1);
-      // one lane waits; the outcome is broadcast so that the warp stays converged for the
-      // .sync.aligned TMEM loads below
-      int ok = 1;
-      if (lane == 0) ok = mbar_wait(&accf_bar[buf], use & 1u, &abort_flag) ? 1 : 0;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      tc_fence_after();
-      const int tm = tile % a.tiles_m, tn = tile / a.tiles_m;
-      const int row = tm * kTcBM + q * 32 + lane;
-      const bool rok = row < a.M;
-      const float scale = rok ? a.s_x[row] * a.alpha : 0.f;
-#pragma unroll 1
-      for (int c = 0; c < kTcBN / 32; ++c) {
-        uint32_t r[32];
-        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kTcBN + c * 32);
-        tmem_ld_32x32b_x32(taddr, r);
-        const int col0 = tn * kTcBN + c * 32;
-        if (rok && col0 < a.N) {
-          const bool full = col0 + 32 <= a.N;
-          if (a.out_bf16) {
-            __nv_bfloat16* yrow = reinterpret_cast<__nv_bfloat16*>(a.Y) + (size_t)row * a.N + col0;
-            if (full) {
-#pragma unroll
-              for (int j = 0; j < 32; j += 8) {
-                uint4 o;
-                uint32_t* op = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                  const __nv_bfloat162 p2 = __floats2bfloat162_rn((float)(int)r[j + 2 * h] * scale,
-                                                                 (float)(int)r[j + 2 * h + 1] * scale);
-                  op[h] = *reinterpret_cast<const uint32_t*>(&p2);
-                }
-                *reinterpret_cast<uint4*>(yrow + j) = o;
-              }
-            } else {
-              for (int j = 0; j < 32 && col0 + j < a.N; ++j) yrow[j] = __float2bfloat16_rn((float)(int)r[j] * scale);
-            }
-          } else {
-            float* yrow = reinterpret_cast<float*>(a.Y) + (size_t)row * a.N + col0;
-            if (full) {
-#pragma unroll
-              for (int j = 0; j < 32; j += 4) {
-                *reinterpret_cast<float4*>(yrow + j) =
-                    make_float4((float)(int)r[j] * scale, (float)(int)r[j + 1] * scale,
-                                (float)(int)r[j + 2] * scale, (float)(int)r[j + 3] * scale);
-              }
-            } else {
-              for (int j = 0; j < 32 && col0 + j < a.N; ++j) yrow[j] = (float)(int)r[j] * scale;
-            }
-          }
-          if (a.acc_debug) {
-            int32_t* drow = a.acc_debug + (size_t)row * a.N + col0;
-            for (int j = 0; j < 32 && col0 + j < a.N; ++j) drow[j] = (int32_t)r[j];
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&acce_bar[buf]);
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem_base) : "memory");
-  }
-}
 
 }  // namespace hbl

@@ -286,26 +286,6 @@ bool make_map_i8(CUtensorMap* map, const void* base, int K, int rows, int box_ro
   return r == CUDA_SUCCESS;
 }
 
-hbl_status run_tc(const void* codes_i8, const int8_t* w_i8, const TcArgs& a0, cudaStream_t s) {
-  CUtensorMap mA, mB;
-  if (!make_map_i8(&mA, codes_i8, a0.K, a0.M, kTcBM)) return HBL_ECUDA;
-  if (!make_map_i8(&mB, w_i8, a0.K, a0.N, kTcBN)) return HBL_ECUDA;
-  TcArgs a = a0;
-  a.tiles_m = (a.M + kTcBM - 1) / kTcBM;
-  a.tiles_n = (a.N + kTcBN - 1) / kTcBN;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const int ntiles = a.tiles_m * a.tiles_n;
-  const int sms = device_sms(dev);
-  const int grid = ntiles < sms ? ntiles : sms;
-  static SmemLimit lim;
-  const cudaError_t e = allow_smem(gemm_tc_kernel, kTcSmem, lim);
-  if (e != cudaSuccess) return cuda_fail(e);
-  gemm_tc_kernel<<<grid, kTcThreads, kTcSmem, s>>>(mA, mB, a);
-  HBL_CHECK_LAUNCH();
-  return HBL_OK;
-}
-
 hbl_status run_tc2(const void* codes_i8, const int8_t* w_i8, const TcArgs& a0, cudaStream_t s) {
   CUtensorMap mA, mB;
   if (!make_map_i8(&mA, codes_i8, a0.K, a0.M, 128)) return HBL_ECUDA;
@@ -407,8 +387,6 @@ hbl_status run_swap(const void* codes_i8, const void* w2, const TcArgs& t, cudaS
 
 // Token counts up to this bound run on CUDA cores (weight bytes bound the product there).
 constexpr int kDecodeMaxM = 8;
-// From this token count on, the product runs on SM pairs (256 x 256 tiles).
-constexpr int kPairMinM = 256;
 
 hbl_status run_gemm(const void* codes, int fmt, int abits, const float* s_x, const void* packed, float alpha,
                     int M, int N, int K, void* Y, int out_dtype, int32_t* acc_debug, cudaStream_t s) {
