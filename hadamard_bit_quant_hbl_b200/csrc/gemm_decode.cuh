@@ -215,6 +215,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) gemm_decode_kernel(const Decod
   const int owner = f / FO, fo = f - owner * FO;
   const uint32_t slot0 = smem_u32(slots);
   cluster_wait();  // every CTA of the cluster is running
+  pdl_launch_dependents();  // the next kernel may launch (it waits for this one before reading Y)
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
     acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], 1);

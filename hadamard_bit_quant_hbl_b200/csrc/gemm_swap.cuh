@@ -21,7 +21,9 @@
 //   warps 2-5  widen each 2-bit row (8 words = 128 codes c = t+1) to 128 int8 t in the
 //              128-byte-swizzled K-major layout the MMA reads (NW-stage ring), then the epilogue:
 //              tcgen05.ld of the partial sums, reduction across the cluster, dequant, store.
-// Every mbarrier wait is bounded (1 s).
+// The kernel may start while the activation kernel before it still runs (programmatic dependent
+// launch): setup, the weight copies and the widening need nothing from it; the activation
+// producer and the epilogue wait for it first. Every mbarrier wait is bounded (1 s).
 #pragma once
 
 #include <cuda.h>
@@ -148,7 +150,9 @@ gemm_swap_kernel(const __grid_constant__ CUtensorMap mapA, const SwapArgs a) {
       }
     }
   } else if (warp == 6) {
-    // ---------------- producer of the activation tiles (runs up to NA ahead)
+    // ---------------- producer of the activation tiles (runs up to NA ahead). The codes may come
+    // from the kernel before this one: wait for it (programmatic dependent launch) first.
+    pdl_wait();
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
@@ -261,6 +265,10 @@ gemm_swap_kernel(const __grid_constant__ CUtensorMap mapA, const SwapArgs a) {
       for (int m = 0; m < Mt; ++m) part[m * kSwNT + (warp & 3) * 32 + lane] = 0;
     }
   }
+
+  // the next kernel of the stream may launch now (it waits for this one before reading Y)
+  pdl_launch_dependents();
+  pdl_wait();  // s_x below comes from the kernel before this one
 
   // ---------------- epilogue part 2: reduce the cluster's partial sums, dequant, store
   __syncwarp();

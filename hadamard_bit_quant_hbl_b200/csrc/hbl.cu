@@ -112,7 +112,18 @@ hbl_status launch_nfq_t(const NfqArgs& a, int threads, int smem, cudaStream_t s)
   // prefetch distance: the groups resident on the device at once (the group that starts when
   // this CTA's successor does)
   b.pf_dist = persistent_grid(k, threads, smem, 1 << 30);
-  k<<<b.groups, threads, smem, s>>>(b);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(b.groups, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may overlap the kernel before
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t le = cudaLaunchKernelEx(&cfg, k, b);
+  if (le != cudaSuccess) return cuda_fail(le);
   HBL_CHECK_LAUNCH();
   return HBL_OK;
 }
@@ -372,13 +383,15 @@ hbl_status run_swap(const void* codes_i8, const void* w2, const TcArgs& t, cudaS
   cfg.blockDim = dim3(kSwThreads, 1, 1);
   cfg.dynamicSmemBytes = kSwSmem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = S;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may overlap the kernel before
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, gemm_swap_kernel, mA, a);
   if (e != cudaSuccess) return cuda_fail(e);
   HBL_CHECK_LAUNCH();

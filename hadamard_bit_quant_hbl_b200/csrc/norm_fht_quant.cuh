@@ -225,8 +225,11 @@ __global__ void __maxnreg__(nfq_max_regs(EB, R)) norm_fht_quant_kernel(const Nfq
   // nothing, so that every load is unconditional.
   const int srow = live_row ? row : a.M - 1;
 
-  // the product that consumes these codes may start now: it streams its weights, which this
-  // kernel does not write, and waits for this kernel's completion before it reads the codes
+  // X may come from the kernel before this one (launched early by programmatic dependent
+  // launch): wait for it. Then the product that consumes these codes may start: it streams its
+  // weights, which this kernel does not write, and waits for this kernel's completion before it
+  // reads the codes.
+  pdl_wait();
   pdl_launch_dependents();
 
   // a later group's rows into L2 while this group loads and computes
