@@ -10,17 +10,22 @@
 //   D[n, m] = sum_k t[k, n] q[m, k],   tcgen05.mma kind::i8, M = 128, N = Mt (16..256), K = 32.
 //
 // A cluster of S CTAs shares one 128-feature tile and splits K: CTA r owns a contiguous run of
-// 128-wide k-blocks. Its partial sums end in its own shared memory and are reduced across the
-// cluster through distributed shared memory, so no global workspace is needed.
+// 128-wide k-blocks, processed in batches of B k-blocks. Its partial sums end in its own shared
+// memory and are reduced across the cluster through distributed shared memory, so no global
+// workspace is needed.
 //
-//   warp 0     TMA producer: per k-block the 2-bit weight tile (4 KB contiguous in the blob's
-//              tile-major section, one bulk copy) and the activation tile (Mt rows x 128 bytes,
-//              128-byte swizzle) into an NL-stage ring.
-//   warp 1     TMEM allocation; one thread issues 4 MMAs per k-block and commits to the ring's
-//              "empty" barriers.
-//   warps 2-5  widen each 2-bit row (8 words = 128 codes c = t+1) to 128 int8 t in the
-//              128-byte-swizzled K-major layout the MMA reads (NW-stage ring), then the epilogue:
-//              tcgen05.ld of the partial sums, reduction across the cluster, dequant, store.
+//   warp 0      bulk copies of the 2-bit weight tiles of a batch (B x 4 KB, contiguous in the
+//               blob's tile-major section) into a 2-stage ring
+//   warp 1      TMEM allocation; one thread issues the batch's B x 4 MMAs and commits once per
+//               batch to the "empty" barriers of the widened tiles and of the activations
+//   warp 2      TMA copies of the batch's activation tiles (Mt rows x 128 bytes per k-block,
+//               128-byte swizzle) into an NA-stage ring
+//   warps 3-10  widen the 2-bit rows (two threads per weight row, 64 codes c = t+1 each) to int8
+//               t in the 128-byte-swizzled K-major layout the MMA reads (2 batch stages), then
+//               the epilogue: tcgen05.ld of the partial sums (warps 3-6), reduction across the
+//               cluster, dequant, store.
+// Synchronisation is per batch, not per k-block: one wait, one proxy fence and one arrive per
+// widening warp and batch (each costs about as much as widening a k-block).
 // The kernel may start while the activation kernel before it still runs (programmatic dependent
 // launch): setup, the weight copies and the widening need nothing from it; the activation
 // producer and the epilogue wait for it first. Every mbarrier wait is bounded (1 s).
@@ -39,11 +44,12 @@ constexpr int kSwNT = 128;        // output features per tile (MMA M)
 constexpr int kSwBK = 128;        // k per block
 constexpr int kSwRaw = 128 * 32;  // bytes of one 2-bit weight tile (4 KB, contiguous in the blob)
 constexpr int kSwWide = 128 * kSwBK;
-constexpr int kSwGR = 4;          // k-blocks per 2-bit copy (16 KB: few, large bulk copies)
-constexpr int kSwNR = 4;          // 2-bit copy stages (released as soon as they are widened)
-constexpr int kSwMaxNA = 8;       // activation copy stages (released by the MMA)
-constexpr int kSwMaxNW = 4;       // widened tile stages (released by the MMA)
-constexpr int kSwThreads = 224;   // 7 warps
+constexpr int kSwNR = 2;          // 2-bit copy stages (one batch each)
+constexpr int kSwNWB = 2;         // widened batch stages
+constexpr int kSwMaxNA = 4;       // activation copy stages (one batch each)
+constexpr int kSwMaxB = 4;        // k-blocks per batch
+constexpr int kSwWidenWarps = 8;
+constexpr int kSwThreads = 32 * (3 + kSwWidenWarps);  // 352
 constexpr int kSwSmem = 200 * 1024 + 1024;
 
 struct SwapArgs {
@@ -52,8 +58,8 @@ struct SwapArgs {
   float alpha;
   int M, N, K;
   int Mt;           // tokens padded to a multiple of 16 (MMA N)
-  int NA, NW;       // activation / widened ring stages
-  int GA;           // k-blocks per activation copy (about 16 KB per copy)
+  int B;            // k-blocks per batch
+  int NA;           // activation ring stages
   int S;            // CTAs per cluster (k split)
   int tmem_cols;
   void* Y;
@@ -81,22 +87,30 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Bounded wait for the last phase armed on a barrier (used only on the abort path, so that no
+// copy is in flight into shared memory when the CTA exits).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < kWaitLimitNs) {
+  }
+}
+
 __global__ void __launch_bounds__(kSwThreads, 1)
 gemm_swap_kernel(const __grid_constant__ CUtensorMap mapA, const SwapArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw3[];
   __shared__ __align__(8) uint64_t raw_full[kSwNR], raw_empty[kSwNR];
   __shared__ __align__(8) uint64_t act_full[kSwMaxNA], act_empty[kSwMaxNA];
-  __shared__ __align__(8) uint64_t wide_full[kSwMaxNW], wide_empty[kSwMaxNW], acc_full, drain_bar;
+  __shared__ __align__(8) uint64_t wide_full[kSwNWB], wide_empty[kSwNWB], acc_full, drain_bar;
   __shared__ uint32_t tmem_base_slot;
   __shared__ volatile int abort_flag;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw3) + 1023) & ~uintptr_t(1023));
-  const int NA = a.NA, NW = a.NW, Mt = a.Mt, GA = a.GA;
+  const int NA = a.NA, Mt = a.Mt, B = a.B;
   const int act_bytes = Mt * kSwBK;                 // one k-block of activations, multiple of 2048
-  const int act_stage = GA * act_bytes;             // one copy: GA k-blocks, [GA][Mt][128] swizzled
+  const int act_stage = B * act_bytes;              // one copy: B k-blocks, [B][Mt][128] swizzled
   uint8_t* act = smem;                              // NA x act_stage
-  uint8_t* wide = act + NA * act_stage;             // NW x 16 KB (128-byte swizzle)
-  uint8_t* raw = wide + NW * kSwWide;               // NR x (GR x 4 KB)
+  uint8_t* wide = act + NA * act_stage;             // kSwNWB x B x 16 KB (128-byte swizzle)
+  uint8_t* raw = wide + kSwNWB * B * kSwWide;       // kSwNR x B x 4 KB
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -106,19 +120,20 @@ gemm_swap_kernel(const __grid_constant__ CUtensorMap mapA, const SwapArgs a) {
   const int KB = a.K / kSwBK;
   const int kb0 = (int)(((long)KB * rank) / S), kb1 = (int)(((long)KB * (rank + 1)) / S);
   const int nkb = kb1 - kb0;
+  const int nbat = (nkb + B - 1) / B;
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int s = 0; s < kSwNR; ++s) {
       mbar_init(&raw_full[s], 1);
-      mbar_init(&raw_empty[s], 4);  // one lane of each widening warp
+      mbar_init(&raw_empty[s], kSwWidenWarps);  // one lane of each widening warp
     }
     for (int s = 0; s < NA; ++s) {
       mbar_init(&act_full[s], 1);
       mbar_init(&act_empty[s], 1);
     }
-    for (int s = 0; s < NW; ++s) {
-      mbar_init(&wide_full[s], 4);
+    for (int s = 0; s < kSwNWB; ++s) {
+      mbar_init(&wide_full[s], kSwWidenWarps);
       mbar_init(&wide_empty[s], 1);
     }
     mbar_init(&acc_full, 1);
@@ -137,57 +152,56 @@ gemm_swap_kernel(const __grid_constant__ CUtensorMap mapA, const SwapArgs a) {
   const uint32_t tmem_base = tmem_base_slot;
 
   if (warp == 0) {
-    // ---------------- producer of the 2-bit weight tiles (runs up to kSwNR ahead)
+    // ---------------- 2-bit weight tiles, one bulk copy per batch (runs up to kSwNR ahead)
     if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0;
-      for (int i = 0; i < nkb; i += kSwGR) {
-        if (!mbar_wait(&raw_empty[s], ph ^ 1u, &abort_flag)) break;
-        const uint32_t bytes = (uint32_t)min(kSwGR, nkb - i) * kSwRaw;  // tiles of one feature tile are consecutive
+      int b = 0;
+      for (; b < nbat; ++b) {
+        const int s = b % kSwNR;
+        if (!mbar_wait(&raw_empty[s], ((uint32_t)(b / kSwNR) & 1u) ^ 1u, &abort_flag)) break;
+        const uint32_t bytes = (uint32_t)min(B, nkb - b * B) * kSwRaw;  // a feature tile's k-blocks are consecutive
         mbar_arrive_expect_tx(&raw_full[s], bytes);
-        bulk_load_1d(raw + s * (kSwGR * kSwRaw), a.w2 + ((size_t)tile * KB + kb0 + i) * 1024, bytes, &raw_full[s]);
-        if (++s == kSwNR) { s = 0; ph ^= 1u; }
+        bulk_load_1d(raw + s * (B * kSwRaw), a.w2 + ((size_t)tile * KB + kb0 + b * B) * 1024, bytes, &raw_full[s]);
       }
+      if (abort_flag)  // no copy may still be landing when the CTA exits
+        for (int d = max(0, b - kSwNR); d < b; ++d) drain_wait(&raw_full[d % kSwNR], (uint32_t)(d / kSwNR) & 1u);
     }
-  } else if (warp == 6) {
-    // ---------------- producer of the activation tiles (runs up to NA ahead). The codes may come
-    // from the kernel before this one: wait for it (programmatic dependent launch) first.
+  } else if (warp == 2) {
+    // ---------------- activation tiles, one TMA copy per batch (runs up to NA ahead). The codes
+    // may come from the kernel before this one: wait for it (programmatic dependent launch).
     pdl_wait();
     if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0;
-      for (int i = 0; i < nkb; i += GA) {
-        if (!mbar_wait(&act_empty[s], ph ^ 1u, &abort_flag)) break;
+      int b = 0;
+      for (; b < nbat; ++b) {
+        const int s = b % NA;
+        if (!mbar_wait(&act_empty[s], ((uint32_t)(b / NA) & 1u) ^ 1u, &abort_flag)) break;
         mbar_arrive_expect_tx(&act_full[s], (uint32_t)act_stage);  // the box is always complete
-        tma_load_3d(act + s * act_stage, &mapA, &act_full[s], 0, 0, kb0 + i);
-        if (++s == NA) { s = 0; ph ^= 1u; }
+        tma_load_3d(act + s * act_stage, &mapA, &act_full[s], 0, 0, kb0 + b * B);
       }
+      if (abort_flag)
+        for (int d = max(0, b - NA); d < b; ++d) drain_wait(&act_full[d % NA], (uint32_t)(d / NA) & 1u);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer
+    // ---------------- MMA issuer: per batch one wait on each ring, B x 4 MMAs, one commit each
     if (lane == 0) {
       const uint32_t idesc = idesc_i8_mn(kSwNT, Mt);
-      int sa = 0, w = 0;
-      uint32_t pha = 0, phw = 0;
       bool ok = true, any = false;
-      for (int i = 0; i < nkb; ++i) {
-        const int ja = i % GA;  // k-block within the activation copy
-        if (!mbar_wait(&wide_full[w], phw, &abort_flag)) { ok = false; break; }
-        if (ja == 0 && !mbar_wait(&act_full[sa], pha, &abort_flag)) { ok = false; break; }
+      for (int b = 0; b < nbat; ++b) {
+        const int ws = b % kSwNWB, as = b % NA;
+        if (!mbar_wait(&wide_full[ws], (uint32_t)(b / kSwNWB) & 1u, &abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&act_full[as], (uint32_t)(b / NA) & 1u, &abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t w_addr = smem_u32(wide + w * kSwWide);
-        const uint32_t a_addr = smem_u32(act + sa * act_stage + ja * act_bytes);
+        const int nb = min(B, nkb - b * B);
+        for (int u = 0; u < nb; ++u) {
+          const uint32_t w_addr = smem_u32(wide + (ws * B + u) * kSwWide);
+          const uint32_t a_addr = smem_u32(act + as * act_stage + u * act_bytes);
 #pragma unroll
-        for (int kk = 0; kk < kSwBK / 32; ++kk)
-          mma_i8(tmem_base, smem_desc_sw128(w_addr + kk * 32), smem_desc_sw128(a_addr + kk * 32), idesc,
-                 (i | kk) != 0 ? 1u : 0u);
-        any = true;
-        mma_commit(&wide_empty[w]);
-        if (ja == GA - 1 || i == nkb - 1) {
-          mma_commit(&act_empty[sa]);
-          if (++sa == NA) { sa = 0; pha ^= 1u; }
+          for (int kk = 0; kk < kSwBK / 32; ++kk)
+            mma_i8(tmem_base, smem_desc_sw128(w_addr + kk * 32), smem_desc_sw128(a_addr + kk * 32), idesc,
+                   (b | u | kk) != 0 ? 1u : 0u);
         }
-        if (++w == NW) { w = 0; phw ^= 1u; }
+        any = true;
+        mma_commit(&wide_empty[ws]);
+        mma_commit(&act_empty[as]);
       }
       if (ok && any) mma_commit(&acc_full);
       if (!ok && any) {
@@ -198,71 +212,61 @@ gemm_swap_kernel(const __grid_constant__ CUtensorMap mapA, const SwapArgs a) {
       }
     }
   } else {
-    // ---------------- widen (warps 2-5, thread = weight row of the tile). A 2-bit tile is released
-    // as soon as it is in registers; the widened tiles of a batch share one proxy fence.
-    const int row = threadIdx.x - 64;  // 0..127
-    const int batch = NW / 2;
-    int s = 0, w = 0;
-    uint32_t ph = 0, phw = 0;
+    // ---------------- widen (warps 3-10): thread (row r, half h) turns the 64 codes of words
+    // 4h..4h+3 of weight row r into four 16-byte chunks of the swizzled int8 row
+    const int tw = threadIdx.x - 96;
+    const int row = tw >> 1, h = tw & 1;
     bool ok = true;
-    for (int i0 = 0; i0 < nkb && ok; i0 += batch) {
-      const int nb = min(batch, nkb - i0);
-      int w1 = w;
-      uint32_t phw1 = phw;
-      for (int j = 0; j < nb; ++j) {
-        // every lane waits (the TMA-written tile must be visible to each reader); the outcome
-        // is made uniform so that the warp stays converged
-        const int i = i0 + j, jr = i % kSwGR;  // k-block within the 2-bit copy
-        bool r = jr != 0 || mbar_wait(&raw_full[s], ph, &abort_flag);
-        if (r) r = mbar_wait(&wide_empty[w1], phw1 ^ 1u, &abort_flag);
-        if (!__all_sync(0xffffffffu, r)) { ok = false; break; }
-        const uint8_t* rp = raw + s * (kSwGR * kSwRaw) + jr * kSwRaw + row * 32;
-        const uint4 lo = *reinterpret_cast<const uint4*>(rp);
-        const uint4 hi = *reinterpret_cast<const uint4*>(rp + 16);
-        if (jr == kSwGR - 1 || i == nkb - 1) {  // the copy is consumed: hand it back
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&raw_empty[s]);
-          if (++s == kSwNR) { s = 0; ph ^= 1u; }
-        }
-        const uint32_t wd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-        uint8_t* dst = wide + w1 * kSwWide + row * 128;
+    for (int b = 0; b < nbat && ok; ++b) {
+      const int rs = b % kSwNR, ws = b % kSwNWB;
+      // every lane waits (the copy-written tile must be visible to each reader); the outcome is
+      // made uniform so that the warp stays converged
+      bool r = mbar_wait(&raw_full[rs], (uint32_t)(b / kSwNR) & 1u, &abort_flag);
+      if (r) r = mbar_wait(&wide_empty[ws], ((uint32_t)(b / kSwNWB) & 1u) ^ 1u, &abort_flag);
+      if (!__all_sync(0xffffffffu, r)) { ok = false; break; }
+      const int nb = min(B, nkb - b * B);
+      for (int u = 0; u < nb; ++u) {
+        const uint4 wv = *reinterpret_cast<const uint4*>(raw + (rs * B + u) * kSwRaw + row * 32 + h * 16);
+        const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+        uint8_t* dst = wide + (ws * B + u) * kSwWide + row * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {  // word c = 16 codes k = 16c + 4s' + b, c' = t + 1 in {0,1,2}
+        for (int i = 0; i < 4; ++i) {  // word 4h+i: 16 codes k = 16(4h+i) + 4s' + b, c' = t + 1 in {0,1,2}
           uint32_t o[4];
 #pragma unroll
           for (int sp = 0; sp < 4; ++sp) {
-            const uint32_t u = (wd[c] >> (2 * sp)) & 0x03030303u;  // c' per byte
-            o[sp] = (u + 0x7f7f7f7fu) ^ 0x80808080u;             // int8 t = c' - 1, no carries
+            const uint32_t u8 = (wd[i] >> (2 * sp)) & 0x03030303u;  // c' per byte
+            o[sp] = (u8 + 0x7f7f7f7fu) ^ 0x80808080u;               // int8 t = c' - 1, no carries
           }
+          const int c = 4 * h + i;
           *reinterpret_cast<uint4*>(dst + ((c ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
         }
-        if (++w1 == NW) { w1 = 0; phw1 ^= 1u; }
       }
-      if (!ok) break;
-      fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
       __syncwarp();
-      for (int j = 0; j < nb; ++j) {
-        if (lane == 0) mbar_arrive(&wide_full[w]);
-        if (++w == NW) { w = 0; phw ^= 1u; }
-      }
+      if (lane == 0) mbar_arrive(&raw_empty[rs]);  // this warp's reads of the 2-bit copy are done
+      fence_proxy_async_smem();                    // generic-proxy writes -> visible to the tensor core
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&wide_full[ws]);
     }
 
     // ---------------- epilogue part 1: partial sums -> own shared memory as [Mt][128] int32
+    // (warps 3-6, one per TMEM lane quarter)
     bool r = ok && mbar_wait(&acc_full, 0, &abort_flag);
     r = __all_sync(0xffffffffu, r);
     int32_t* part = reinterpret_cast<int32_t*>(smem);  // the rings are idle now
-    if (r && nkb > 0) {
-      tc_fence_after();
+    if (warp <= 6) {
       const int q = warp & 3;  // TMEM lane quarter
       const int f = q * 32 + lane;
-      for (int c0 = 0; c0 < Mt; c0 += 16) {
-        uint32_t v[16];
-        tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+      if (r && nkb > 0) {
+        tc_fence_after();
+        for (int c0 = 0; c0 < Mt; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) part[(c0 + j) * kSwNT + f] = (int32_t)v[j];
+          for (int j = 0; j < 16; ++j) part[(c0 + j) * kSwNT + f] = (int32_t)v[j];
+        }
+      } else {
+        for (int m = 0; m < Mt; ++m) part[m * kSwNT + f] = 0;
       }
-    } else {
-      for (int m = 0; m < Mt; ++m) part[m * kSwNT + (warp & 3) * 32 + lane] = 0;
     }
   }
 
@@ -274,10 +278,11 @@ gemm_swap_kernel(const __grid_constant__ CUtensorMap mapA, const SwapArgs a) {
   __syncwarp();
   tc_fence_before();
   cluster_sync_all();
-  if (warp >= 2 && warp <= 5) {
+  if (warp >= 3) {
     const uint32_t part0 = smem_u32(smem);
-    const int t = threadIdx.x - 64;
-    for (int e = (int)rank * 128 + t; e < Mt * kSwNT; e += S * 128) {
+    const int t = threadIdx.x - 96;
+    const int nt = 32 * kSwWidenWarps;
+    for (int e = (int)rank * nt + t; e < Mt * kSwNT; e += S * nt) {
       const int m = e / kSwNT, f = e - m * kSwNT;
       const int n = n0 + f;
       if (m >= a.M || n >= a.N) continue;

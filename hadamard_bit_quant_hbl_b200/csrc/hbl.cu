@@ -351,12 +351,13 @@ hbl_status run_swap(const void* codes_i8, const void* w2, const TcArgs& t, cudaS
   a.N = t.N;
   a.K = t.K;
   a.Mt = (t.M + 15) / 16 * 16;
-  // activation copies of about 16 KB; shared memory: 4 x 16 KB of 2-bit tiles, NW x 16 KB
-  // widened tiles, the rest activation copies
-  a.GA = a.Mt >= 128 ? 1 : 128 / a.Mt;
-  a.NW = a.Mt <= 128 ? kSwMaxNW : 3;
-  a.NA = (200 * 1024 - kSwNR * kSwGR * kSwRaw - a.NW * kSwWide) / (a.GA * a.Mt * kSwBK);
+  // batches of B k-blocks (fewer for wide activation tiles); shared memory: 2 batch stages of
+  // widened tiles (B x 16 KB each), 2 of 2-bit tiles (B x 4 KB), the rest activation copies of
+  // one batch each (B x Mt x 128 bytes)
+  a.B = a.Mt <= 32 ? 4 : (a.Mt <= 128 ? 2 : 1);
+  a.NA = (200 * 1024 - a.B * (kSwNWB * kSwWide + kSwNR * kSwRaw)) / (a.B * a.Mt * kSwBK);
   if (a.NA > kSwMaxNA) a.NA = kSwMaxNA;
+  if (a.NA < 1) return HBL_EUNSUPPORTED;  // not reached for Mt <= 256
   int cols = 32;
   while (cols < a.Mt) cols *= 2;
   a.tmem_cols = cols;
@@ -374,7 +375,7 @@ hbl_status run_swap(const void* codes_i8, const void* w2, const TcArgs& t, cudaS
   a.S = S;
   a.w2 = static_cast<const uint32_t*>(w2);
   CUtensorMap mA;
-  if (!make_map_i8_blocks(&mA, codes_i8, a.K, a.M, a.Mt, a.GA)) return HBL_ECUDA;
+  if (!make_map_i8_blocks(&mA, codes_i8, a.K, a.M, a.Mt, a.B)) return HBL_ECUDA;
   static SmemLimit lim;
   cudaError_t e = allow_smem(gemm_swap_kernel, kSwSmem, lim);
   if (e != cudaSuccess) return cuda_fail(e);
