@@ -47,7 +47,7 @@ NCU_TRAFFIC = {
 
 def product_kernel(M):
     """Name and source file of the product kernel hbl_ternary_gemm runs for M tokens."""
-    if M <= 8:
+    if M <= 4:
         return "gemm_decode", "gemm_decode.cuh"
     return ("gemm_swap", "gemm_swap.cuh") if M <= 256 else ("gemm_tc2", "gemm_tc2.cuh")
 

@@ -24,6 +24,10 @@
 //               t in the 128-byte-swizzled K-major layout the MMA reads (2 batch stages), then
 //               the epilogue: tcgen05.ld of the partial sums (warps 3-6), reduction across the
 //               cluster, dequant, store.
+// The rings take 200 KB (batches of 4 up to 32 tokens, 2 up to 128, else 1), one CTA per SM; the
+// partial sums ([Mt][128] int32) reuse them in the epilogue. (Two 100 KB CTAs per SM are faster
+// for a lone product but slow the forward pass down: they share SMs with the activation kernel
+// that runs before them, whose rows are its critical path.)
 // Synchronisation is per batch, not per k-block: one wait, one proxy fence and one arrive per
 // widening warp and batch (each costs about as much as widening a k-block).
 // The kernel may start while the activation kernel before it still runs (programmatic dependent
@@ -47,10 +51,9 @@ constexpr int kSwWide = 128 * kSwBK;
 constexpr int kSwNR = 2;          // 2-bit copy stages (one batch each)
 constexpr int kSwNWB = 2;         // widened batch stages
 constexpr int kSwMaxNA = 4;       // activation copy stages (one batch each)
-constexpr int kSwMaxB = 4;        // k-blocks per batch
 constexpr int kSwWidenWarps = 8;
 constexpr int kSwThreads = 32 * (3 + kSwWidenWarps);  // 352
-constexpr int kSwSmem = 200 * 1024 + 1024;
+constexpr int kSwSmem = 200 * 1024;  // ring budget, one CTA per SM
 
 struct SwapArgs {
   const uint32_t* w2;  // 2-bit weight section, tile-major (4 KB per 128 x 128 tile)

@@ -355,7 +355,7 @@ hbl_status run_swap(const void* codes_i8, const void* w2, const TcArgs& t, cudaS
   // widened tiles (B x 16 KB each), 2 of 2-bit tiles (B x 4 KB), the rest activation copies of
   // one batch each (B x Mt x 128 bytes)
   a.B = a.Mt <= 32 ? 4 : (a.Mt <= 128 ? 2 : 1);
-  a.NA = (200 * 1024 - a.B * (kSwNWB * kSwWide + kSwNR * kSwRaw)) / (a.B * a.Mt * kSwBK);
+  a.NA = (kSwSmem - a.B * (kSwNWB * kSwWide + kSwNR * kSwRaw)) / (a.B * a.Mt * kSwBK);
   if (a.NA > kSwMaxNA) a.NA = kSwMaxNA;
   if (a.NA < 1) return HBL_EUNSUPPORTED;  // not reached for Mt <= 256
   int cols = 32;
@@ -377,12 +377,13 @@ hbl_status run_swap(const void* codes_i8, const void* w2, const TcArgs& t, cudaS
   CUtensorMap mA;
   if (!make_map_i8_blocks(&mA, codes_i8, a.K, a.M, a.Mt, a.B)) return HBL_ECUDA;
   static SmemLimit lim;
-  cudaError_t e = allow_smem(gemm_swap_kernel, kSwSmem, lim);
+  const int smem = kSwSmem + 1024;  // + alignment slack
+  cudaError_t e = allow_smem(gemm_swap_kernel, smem, lim);
   if (e != cudaSuccess) return cuda_fail(e);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ntiles * S, 1, 1);
   cfg.blockDim = dim3(kSwThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSwSmem;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -399,15 +400,18 @@ hbl_status run_swap(const void* codes_i8, const void* w2, const TcArgs& t, cudaS
   return HBL_OK;
 }
 
-// Token counts up to this bound run on CUDA cores (weight bytes bound the product there).
-constexpr int kDecodeMaxM = 8;
+// Token counts up to these bounds run on CUDA cores (weight bytes bound the product there):
+// int8 codes up to 4 tokens (from 5 on the swapped tensor-core kernel is faster), packed int4
+// codes up to 8 (the tensor-core kernels read one int8 per code).
+constexpr int kDecodeMaxM = 4;
+constexpr int kDecodeMaxMPacked = 8;
 
 hbl_status run_gemm(const void* codes, int fmt, int abits, const float* s_x, const void* packed, float alpha,
                     int M, int N, int K, void* Y, int out_dtype, int32_t* acc_debug, cudaStream_t s) {
   const BlobLayout bl = blob_layout(K, N);
   const uint8_t* blob = static_cast<const uint8_t*>(packed);
   const bool packed4 = (abits == 4 && fmt == HBL_CODES_PACKED);
-  if (M <= kDecodeMaxM) {
+  if (M <= (packed4 ? kDecodeMaxMPacked : kDecodeMaxM)) {
     DecodeArgs d;
     d.m0 = 0;
     d.codes = static_cast<const uint8_t*>(codes);

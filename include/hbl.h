@@ -151,9 +151,13 @@ hbl_status hbl_norm_fht_quant(const void* X, const float* gain, int M, int K, in
  *   packed   blob from hbl_pack_weights / hbl_pack_ternary for this K, N
  *   Y        device [M][N] of out_dtype (fp32 or bf16), 16-byte aligned, N a multiple of 8
  *   acc_debug  device int32 [M][N] receiving the exact integer sums, or NULL
- * Small M runs on CUDA cores over the 2-bit section; large M on tcgen05 int8 tensor cores
- * over the int8 section (which then needs fmt = HBL_CODES_I8 or abits = 8).
- * Asynchronous. */
+ * Kernels by token count (int8 codes): M <= 4 on CUDA cores and 5 <= M <= 256 on tcgen05
+ * tensor cores, both over the 2-bit section; M > 256 on tcgen05 SM pairs over the int8
+ * section. Packed int4 codes (fmt = HBL_CODES_PACKED with abits = 4) are taken by the CUDA-core
+ * kernel only: M <= 8, else HBL_EUNSUPPORTED.
+ * Asynchronous. The kernel may begin streaming weights before the kernel before it in the
+ * stream has finished, and waits for that kernel before it reads codes or s_x; Y must not alias
+ * the inputs of the kernel before it. */
 hbl_status hbl_ternary_gemm(const void* codes, hbl_codes_fmt fmt, int abits, const float* s_x,
                             const void* packed, size_t packed_bytes, float alpha, int M, int N,
                             int K, void* Y, hbl_out_dtype out_dtype, int32_t* acc_debug,

@@ -185,8 +185,8 @@ def run_gemm_with_oracle_codes(q, t, s, alpha, fmt, abits):
 
 
 GEMM_CASES = [
-    # (M, K, N, abits, fmt)  -- M <= 8 runs on CUDA cores, up to 256 on swapped tcgen05 tiles,
-    # larger M on SM pairs
+    # (M, K, N, abits, fmt)  -- int8 codes: M <= 4 on CUDA cores, up to 256 on swapped tcgen05
+    # tiles, larger M on SM pairs; packed int4 codes: M <= 8 on CUDA cores
     (1, 256, 8, 4, hbl.HBL_CODES_PACKED),
     (1, 16384, 264, 4, hbl.HBL_CODES_PACKED),
     (2, 4096, 128, 8, hbl.HBL_CODES_PACKED),
