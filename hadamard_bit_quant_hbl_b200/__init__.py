@@ -20,7 +20,7 @@ __all__ = [
     "HBL_Q_A8_ABSMAX", "HBL_Q_A4_ABSMEAN", "HBL_Q_A4_ABSMAX",
     "HBL_CODES_PACKED", "HBL_CODES_I8", "HBL_OUT_F32", "HBL_OUT_BF16",
     "HblError", "lib", "library_path",
-    "hbl_status_string", "hbl_device_status", "hbl_packed_weights_bytes", "hbl_pack_weights_workspace",
+    "hbl_status_string", "hbl_device_status", "hbl_selftest_timeout", "hbl_packed_weights_bytes", "hbl_pack_weights_workspace",
     "hbl_pack_weights", "hbl_pack_ternary", "hbl_norm_fht_quant", "hbl_ternary_gemm",
     "hbl_forward_workspace", "hbl_forward", "codes_row_bytes",
 ]
@@ -45,6 +45,7 @@ _SIGNATURES = {
     "hbl_status_string": (ctypes.c_char_p, [_c_int]),
     "hbl_last_cuda_error": (_c_int, []),
     "hbl_device_status": (_c_int, [_c_void_p]),
+    "hbl_selftest_timeout": (_c_int, [_c_int, _c_void_p]),
     "hbl_packed_weights_bytes": (_c_size_t, [_c_int, _c_int]),
     "hbl_pack_weights_workspace": (_c_size_t, [_c_int, _c_int]),
     "hbl_pack_weights": (_c_int, [_c_void_p, _c_int, _c_int, _c_float, _c_void_p, _c_size_t,
@@ -124,6 +125,15 @@ def hbl_device_status(stream=None) -> int:
 
     s = torch.cuda.current_stream().cuda_stream if stream is None else _stream(stream, None)
     return lib().hbl_device_status(s)
+
+
+def hbl_selftest_timeout(limit_ms: int = 50, stream=None) -> None:
+    """Launch the time-out self-test kernel (its wait runs out after `limit_ms`); the next
+    hbl_device_status() reports HBL_ETIMEOUT."""
+    import torch
+
+    s = torch.cuda.current_stream().cuda_stream if stream is None else _stream(stream, None)
+    _check(lib().hbl_selftest_timeout(int(limit_ms), s), "hbl_selftest_timeout")
 
 
 def hbl_packed_weights_bytes(K: int, N: int) -> int:

@@ -76,6 +76,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Self-test of the time-out path: one thread waits on a barrier that nothing completes, with the
+// bounded loop of mbar_wait but a short limit; the wait runs out and raises the error flag.
+__global__ void selftest_timeout_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(&bar, 0)) {
+      if (globaltimer_ns() - t0 > limit_ns) {
+        raise_error(kErrTimeout);
+        break;
+      }
+    }
+  }
+}
+
 // 1-D bulk copy global -> shared (TMA engine), completion counted in bytes on `bar`.
 __device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"

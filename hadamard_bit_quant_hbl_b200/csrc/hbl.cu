@@ -482,6 +482,13 @@ hbl_status hbl_device_status(hbl_stream_t stream) {
   return HBL_OK;
 }
 
+hbl_status hbl_selftest_timeout(int limit_ms, hbl_stream_t stream) {
+  if (limit_ms < 1 || limit_ms > 1000) return HBL_EINVAL;
+  selftest_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>((uint64_t)limit_ms * 1000000ull);
+  HBL_CHECK_LAUNCH();
+  return HBL_OK;
+}
+
 size_t hbl_packed_weights_bytes(int K, int N) {
   if (K <= 0 || N <= 0) return 0;
   return blob_layout(K, N).total;

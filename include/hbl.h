@@ -74,6 +74,14 @@ int hbl_last_cuda_error(void);
  * call, HBL_OK otherwise (or HBL_ECUDA if the synchronisation itself failed). */
 hbl_status hbl_device_status(hbl_stream_t stream);
 
+/* Diagnostic of the time-out path. Launches on `stream` one small kernel that waits on a
+ * barrier nothing ever completes, with the bounded wait every kernel of this library uses but a
+ * limit of `limit_ms` milliseconds (1 ... 1000) instead of 1 s: the wait runs out, raises the
+ * device error flag and the kernel returns. The next hbl_device_status() then reports
+ * HBL_ETIMEOUT, and the context stays usable. Asynchronous. HBL_EINVAL for a limit outside
+ * the range. */
+hbl_status hbl_selftest_timeout(int limit_ms, hbl_stream_t stream);
+
 /* ---------------------------------------------------------------------------------------
  * Packed ternary weights.
  *

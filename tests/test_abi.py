@@ -108,6 +108,12 @@ def test_pack_rejects_bad_arguments(L):
     assert L.hbl_pack_ternary(FAKE, 512, 63, FAKE, nbytes, None) == hbl.HBL_EINVAL
 
 
+def test_selftest_timeout_rejects_limits_outside_range(L):
+    # checked on the host before any launch
+    assert L.hbl_selftest_timeout(0, None) == hbl.HBL_EINVAL
+    assert L.hbl_selftest_timeout(1001, None) == hbl.HBL_EINVAL
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(hbl, "_lib", None)
     monkeypatch.setattr(hbl, "library_path", str(tmp_path / "nope.so"))
