@@ -293,8 +293,8 @@ def test_forward_small(name, M):
 
 
 FULL = [("single_a8_16x256", None), ("wo_1p3b_a4", None), ("wdown_3b_a4", None), ("wo_7b_a4", 8192),
-        ("wdown_7b_a4", 8192), ("wo_7b_a4", 1), ("wdown_7b_a4", 16), ("wdown_7b_a4", 64), ("wdown_7b_a4", 512),
-        ("wdown_nonpow2_a4", None)]
+        ("wdown_7b_a4", 8192), ("wo_7b_a4", 1), ("wdown_7b_a4", 1), ("wdown_7b_a4", 16), ("wo_7b_a4", 64),
+        ("wdown_7b_a4", 64), ("wdown_7b_a4", 512), ("wdown_nonpow2_a4", None)]
 
 
 @pytest.mark.parametrize("name,M", FULL)
@@ -304,3 +304,27 @@ def test_forward_full_size_sampled_rows(name, M):
     picks = [0, 1, spec.M // 2, spec.M - 1] + list(np.random.default_rng(spec.M).integers(0, spec.M, 4))
     rows = sorted(set(int(r) for r in picks if r < spec.M))
     check_forward(spec, rows=rows, out_dtype=hbl.HBL_OUT_BF16)
+
+
+@pytest.mark.parametrize("M", [1, 3, 16, 64, 300])
+def test_chained_layers_read_the_previous_output(M):
+    # Two layers on one stream, the second fed by the first's output: the second layer's kernels
+    # may launch before the first layer's product has finished (programmatic dependent launch)
+    # and must wait for it before reading. Every kernel reduces in a fixed order, so the result
+    # equals, bit for bit, the second layer run after an explicit synchronisation.
+    spec = inputs.WORKLOADS["wo_7b_a4"].with_m(M)
+    X = to_dev_bf16(inputs.activations(spec))
+    W1 = inputs.weights(spec)
+    W2 = np.ascontiguousarray(W1[::-1, ::-1])
+    p1, a1 = hbl.hbl_pack_weights(torch.from_numpy(W1).cuda())
+    p2, a2 = hbl.hbl_pack_weights(torch.from_numpy(W2).cuda())
+    q = hbl.HBL_Q_A4_ABSMEAN
+    Y1 = hbl.hbl_forward(X, p1, a1, spec.N, None, 0, q, out_dtype=hbl.HBL_OUT_BF16)
+    Y2 = hbl.hbl_forward(Y1, p2, a2, spec.N, None, 0, q, out_dtype=hbl.HBL_OUT_F32)
+    torch.cuda.synchronize()
+    Y1c = Y1.clone()
+    torch.cuda.synchronize()
+    Y2_ref = hbl.hbl_forward(Y1c, p2, a2, spec.N, None, 0, q, out_dtype=hbl.HBL_OUT_F32)
+    torch.cuda.synchronize()
+    assert torch.equal(Y2, Y2_ref)
+    assert hbl.hbl_device_status() == hbl.HBL_OK
