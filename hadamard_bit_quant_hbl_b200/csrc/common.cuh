@@ -93,6 +93,12 @@ __global__ void selftest_timeout_kernel(uint64_t limit_ns) {
   }
 }
 
+// Orders this thread's generic-proxy shared-memory writes before later async-proxy reads (TMA,
+// tensor-core operands).
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // 1-D bulk copy global -> shared (TMA engine), completion counted in bytes on `bar`.
 __device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"

@@ -15,6 +15,7 @@
 #include "gemm_tc2.cuh"
 #include "gemm_swap.cuh"
 #include "norm_fht_quant.cuh"
+#include "norm_fht_quant_tc.cuh"
 #include "pack_weights.cuh"
 
 using namespace hbl;
@@ -144,6 +145,29 @@ constexpr int eb_for(int L) {
   return L == 8 ? 4 : L == 9 ? 5 : L == 10 ? 5 : L == 11 ? 6 : L == 12 ? 6 : 7;
 }
 
+// The 16384-wide transform with the H_128 factor on the tensor cores (no gain, one block).
+template <int QM>
+hbl_status launch_nfq_tc(const NfqArgs& a, cudaStream_t s) {
+  static SmemLimit lim;
+  auto* k = norm_fht_quant_tc_kernel<QM>;
+  cudaError_t e = allow_smem(k, kNtSmem, lim);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(persistent_grid(k, kNtThreads, kNtSmem, a.M), 1, 1);
+  cfg.blockDim = dim3(kNtThreads, 1, 1);
+  cfg.dynamicSmemBytes = kNtSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may overlap the kernel before
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, k, a);
+  if (e != cudaSuccess) return cuda_fail(e);
+  HBL_CHECK_LAUNCH();
+  return HBL_OK;
+}
+
 hbl_status run_nfq(const void* X, const float* gain, int M, int K, int had_block, int quant, float eps_norm,
                    float eps_q, int fmt, void* codes, float* s_x, cudaStream_t stream) {
   const int n = had_block == 0 ? K : had_block;
@@ -189,6 +213,11 @@ hbl_status run_nfq(const void* X, const float* gain, int M, int K, int had_block
   a.groups = (M + rows - 1) / rows;
   a.pf_dist = 0;
 
+  if (L == 14 && nb == 1 && gain == nullptr) {
+    if (quant == 0) return launch_nfq_tc<0>(a, stream);
+    if (quant == 1) return launch_nfq_tc<1>(a, stream);
+    return launch_nfq_tc<2>(a, stream);
+  }
   // K <= 32768 bounds nb, so these R always suffice: L=8 nb<=128 (R<=4), L=9..12 R<=2, L>=13 R=1
   switch (L) {
     case 8:
