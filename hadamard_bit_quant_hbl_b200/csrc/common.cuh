@@ -33,6 +33,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
 }
 
+// The dynamic shared-memory base rounded up to a multiple of A bytes. The offset is added to the
+// shared pointer itself: a round trip through an integer would hide from the compiler that the
+// result addresses shared memory, and every access through it would become a generic one.
+template <uint32_t A>
+__device__ __forceinline__ uint8_t* align_shared(uint8_t* base) {
+  static_assert((A & (A - 1)) == 0, "power of two");
+  return base + ((A - (smem_u32(base) & (A - 1))) & (A - 1));
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
 }

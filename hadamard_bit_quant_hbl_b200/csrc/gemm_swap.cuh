@@ -107,7 +107,7 @@ gemm_swap_kernel(const __grid_constant__ CUtensorMap mapA, const SwapArgs a) {
   __shared__ uint32_t tmem_base_slot;
   __shared__ volatile int abort_flag;
 
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw3) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_shared<1024>(smem_raw3);
   const int NA = a.NA, Mt = a.Mt, B = a.B;
   const int act_bytes = Mt * kSwBK;                 // one k-block of activations, multiple of 2048
   const int act_stage = B * act_bytes;              // one copy: B k-blocks, [B][Mt][128] swizzled

@@ -100,7 +100,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
   __shared__ uint32_t tmem_base_slot;
   __shared__ volatile int abort_flag;
 
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw2) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_shared<1024>(smem_raw2);
   uint8_t* smA = smem;
   uint8_t* smB = smem + kT2Stages * kT2StageA;
 

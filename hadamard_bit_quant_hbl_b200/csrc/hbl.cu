@@ -67,7 +67,12 @@ cudaError_t allow_smem(F* kernel, int bytes, SmemLimit& lim) {
   dev &= 63;
   std::lock_guard<std::mutex> lk(lim.mu);
   if (lim.allowed[dev] >= bytes) return cudaSuccess;
-  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  // the kernels stream their data, so L1 matters less than shared memory: ask for the largest
+  // carveout, so that the occupancy query (which sizes the persistent grids) and the launch agree
+  // on how many CTAs share an SM
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess) lim.allowed[dev] = bytes;
   return e;
 }
@@ -153,7 +158,10 @@ hbl_status launch_nfq_tc(const NfqArgs& a, cudaStream_t s) {
   cudaError_t e = allow_smem(k, kNtSmem, lim);
   if (e != cudaSuccess) return cuda_fail(e);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(persistent_grid(k, kNtThreads, kNtSmem, a.M), 1, 1);
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int resident = kNtCtasPerSm * device_sms(dev);
+  cfg.gridDim = dim3(a.M < resident ? a.M : resident, 1, 1);
   cfg.blockDim = dim3(kNtThreads, 1, 1);
   cfg.dynamicSmemBytes = kNtSmem;
   cfg.stream = s;

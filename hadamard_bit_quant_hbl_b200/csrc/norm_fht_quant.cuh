@@ -384,10 +384,11 @@ __global__ void __maxnreg__(nfq_max_regs(EB, R)) norm_fht_quant_kernel(const Nfq
   }
   if (live_row && tr == 0) a.s_x[row] = sx;
 
-  // ---- 5. codes: fp32 product, clamp (absmean only: absmax products already lie in
-  // [-Q, Q]), then round to nearest even by adding 1.5 * 2^23 -- the integer lands in the low
-  // mantissa bits and, being small, its low 16 bits are the int16 code. 4 codes per word,
-  // 16 bytes per store, into a byte matrix [k mod 8][k / 8].
+  // ---- 5. codes: fma(y, mult, 1.5 * 2^23) rounds the exact product to the nearest integer
+  // (ties to even) in one step, the integer landing in the low mantissa bits (|y mult| < 2^22);
+  // absmean then clamps that integer-valued sum to 1.5 * 2^23 + [-8, 7], exactly (absmax
+  // products already lie in [-Q, Q]). The low byte is the code. 4 codes per word, 16 bytes per
+  // store, into a byte matrix [k mod 8][k / 8].
   const float2 mult2 = make_float2(mult, mult);
   const float2 magic2 = make_float2(12582912.f, 12582912.f);
 #pragma unroll
@@ -406,16 +407,15 @@ __global__ void __maxnreg__(nfq_max_regs(EB, R)) norm_fht_quant_kernel(const Nfq
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int r0 = (x << S2) + j + 4 * q;  // 4 consecutive registers = 2 float2
-            float2 t0 = __fmul2_rn(v[rho][r0 / 2], mult2);
-            float2 t1 = __fmul2_rn(v[rho][r0 / 2 + 1], mult2);
+            float2 p0 = __ffma2_rn(v[rho][r0 / 2], mult2, magic2);
+            float2 p1 = __ffma2_rn(v[rho][r0 / 2 + 1], mult2, magic2);
             if constexpr (!kAbsmax) {
-              t0.x = fminf(fmaxf(t0.x, (float)kLo), (float)kHi);
-              t0.y = fminf(fmaxf(t0.y, (float)kLo), (float)kHi);
-              t1.x = fminf(fmaxf(t1.x, (float)kLo), (float)kHi);
-              t1.y = fminf(fmaxf(t1.y, (float)kLo), (float)kHi);
+              constexpr float lo = 12582912.f + kLo, hi = 12582912.f + kHi;
+              p0.x = fminf(fmaxf(p0.x, lo), hi);
+              p0.y = fminf(fmaxf(p0.y, lo), hi);
+              p1.x = fminf(fmaxf(p1.x, lo), hi);
+              p1.y = fminf(fmaxf(p1.y, lo), hi);
             }
-            const float2 p0 = __fadd2_rn(t0, magic2);
-            const float2 p1 = __fadd2_rn(t1, magic2);
             const uint32_t h0 = __byte_perm(__float_as_uint(p0.x), __float_as_uint(p0.y), 0x5410);
             const uint32_t h1 = __byte_perm(__float_as_uint(p1.x), __float_as_uint(p1.y), 0x5410);
             wds[q] = __byte_perm(h0, h1, 0x6420);

@@ -5,30 +5,31 @@
 // Hadamard transform of the normalised activations before per-token quantisation; the page
 // defines the transform as a matrix product computed with the fast Hadamard transform.
 //
-// H_16384 = H_128 (x) H_128 in Sylvester order: with the index k split into the 7 bits
-// a = (k bits 13..10, k bits 2..0) and the 7 bits n = k bits 9..3,
+// H_16384 = H_128 (x) H_128 in Sylvester order: H[k][k'] = (-1)^popcount(k & k') factors over
+// any split of the 14 index bits. Split k into the 7 bits a = (k bits 13..10, 5..3) and the 7
+// bits n = (k bits 9..6, 2..0):
 //   y[a, n] = sum_{a'} H_128[a][a'] * sum_{n'} H_128[n][n'] * x[a', n'],
 // and the two factors commute. On CUDA cores the 14 butterfly stages cost 14 fp32 adds per
 // element and bound the kernel by the FP32 pipe and issue, not by HBM; here the factor over a is
 // one exact tensor-core product per row,
 //   D[a][n] = sum_{a'} H_128[a][a'] * x[a', n]    (tcgen05.mma kind::f16, bf16 x bf16 -> fp32),
 // exact up to fp32 rounding since x is bf16 and H is +-1, and the factor over n is 7 butterfly
-// stages on CUDA cores. The MMA's B operand is the bf16 row itself, as the TMA copy lands it:
-// 8 consecutive features (k bits 2..0) are one 16-byte row of an 8 x 16-byte core matrix whose
-// 8 rows are 8 consecutive n (16 bytes apart), so the K-major no-swizzle layout reads the row with
-// core matrices 128 bytes apart along N and 2048 bytes apart along K. TMEM lane a of the
-// accumulator then holds, in its 128 columns, exactly the values one thread needs for the
-// remaining stages: no widening pass and no regrouping through shared memory.
+// stages on CUDA cores. The MMA's B operand is the bf16 row itself, as the TMA copy lands it,
+// read MN-major: the 128 contiguous bytes of features 64j .. 64j + 63 are one 8 x 16-byte core
+// matrix whose 16-byte rows hold 8 consecutive n (k bits 2..0) and step through a' (k bits
+// 5..3); core matrices lie 128 bytes apart along N (k bits 9..6) and 2048 bytes apart along K
+// (k bit 10). TMEM lane a of the accumulator then holds, in its 128 columns, exactly the values
+// one thread needs for the remaining stages, and after them 16 runs of 8 consecutive outputs:
+// the thread forms its codes and stores them to global memory directly, with no regrouping
+// through shared memory.
 //
 //   warps 0-3  consumers, thread = TMEM lane a: tcgen05.ld of the 128 columns, 7 butterfly
-//              stages, row statistics, quantisation, codes through a [k mod 8][k / 8] byte matrix
-//              and out in natural order (as the CUDA-core kernel)
+//              stages, row statistics (one named barrier), quantisation, 16 stores of 8 codes
 //   warp 4     TMEM allocation; one thread copies rows in (one 32 KB bulk copy each) and issues
 //              the 8 MMAs (K = 16 each) of a row into one of two TMEM accumulators
-// Persistent CTAs (two per SM) walk the rows. (A 6-slot ring of quarter-row copies with separate
-// copy and MMA threads measured slower: the consumers, 8 warps per SM at 168 registers, are the
-// limit, not the copies.) Every mbarrier wait is bounded (1 s); the
-// consumers vote on the outcome of their waits so that they leave their loop together.
+// Persistent CTAs (two per SM) walk the rows. (With the consumers' arithmetic taken out the copies
+// and MMAs alone run at 5.2 TB/s: the consumers are the limit.) Every mbarrier wait is bounded
+// (1 s); the consumers vote on the outcome of their waits so that they leave their loop together.
 #pragma once
 
 #include "common.cuh"
@@ -41,11 +42,26 @@ constexpr int kNtN = 16384;                       // transform size (the whole r
 constexpr int kNtRowBytes = kNtN * 2;             // one bf16 row
 constexpr int kNtThreads = 160;                   // 4 consumer warps + 1 copy / MMA warp
 constexpr int kNtTmemCols = 256;                  // two 128-column fp32 accumulators
-constexpr int kNtCrow = kNtN / 8 + 16;            // byte stride of a (k mod 8) row of the code matrix
-constexpr int kNtSmem = 32768 + kNtRowBytes + 8 * kNtCrow + 1024;  // H, row, codes, alignment slack
+#ifndef HBL_NT_PAD
+#define HBL_NT_PAD 0
+#endif
+constexpr int kNtSmem = 32768 + kNtRowBytes + HBL_NT_PAD + 1024;  // H, row, alignment slack
+// CTAs resident on one SM. The copy and the MMAs of one CTA overlap the butterflies of the other,
+// so the launch sizes its grid to this many per SM. The register file is split into four
+// 16384-entry quarters, one per warp scheduler, and two 5-warp CTAs put three warps on one quarter:
+// that fits at kNtMaxRegs registers a thread, the count the compiler keeps to under the kernel's
+// launch bounds. (The runtime's occupancy query answers 1 for this kernel, so the launch does not
+// use it.)
+constexpr int kNtCtasPerSm = 2;
+constexpr int kNtMaxRegs = 168;
+static_assert(kNtCtasPerSm * (kNtSmem + 1024) <= 228 * 1024, "shared memory of the resident CTAs");
+static_assert(kNtCtasPerSm * kNtTmemCols <= 512, "TMEM columns of the resident CTAs");
+static_assert((kNtCtasPerSm * kNtThreads / 32 + 3) / 4 * 32 * kNtMaxRegs <= 16384,
+              "registers of the warps the resident CTAs put on one scheduler");
 
-// Shared-memory matrix descriptor: K-major, no swizzle, 8 x 16-byte core matrices `lbo` bytes
-// apart along K and `sbo` bytes apart along M/N.
+// Shared-memory matrix descriptor, no swizzle: 8 x 16-byte core matrices (128 contiguous bytes)
+// `lbo` bytes apart along K and `sbo` bytes apart along M/N. (Whether the 16-byte rows of a core
+// matrix run along K or along M/N is the operand's major-ness in the instruction descriptor.)
 __device__ __forceinline__ uint64_t smem_desc_none(uint32_t addr, uint32_t lbo, uint32_t sbo) {
   uint64_t d = 0;
   d |= (uint64_t)((addr >> 4) & 0x3fffu);
@@ -55,11 +71,12 @@ __device__ __forceinline__ uint64_t smem_desc_none(uint32_t addr, uint32_t lbo, 
   return d;
 }
 
-// Instruction descriptor: kind::f16 with bf16 A and B, fp32 D, both K-major.
+// Instruction descriptor: kind::f16 with bf16 A and B, fp32 D; A K-major, B MN-major.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
   return (1u << 4)                      // D format: f32
          | (1u << 7)                    // A: bf16
          | (1u << 10)                   // B: bf16
+         | (1u << 16)                   // B: MN-major (A stays K-major)
          | ((uint32_t)(N >> 3) << 17)   // N / 8
          | ((uint32_t)(M >> 4) << 24);  // M / 16
 }
@@ -90,20 +107,77 @@ __device__ __forceinline__ bool consumer_bar_or(bool pred) {
   return r != 0;
 }
 
+__device__ __forceinline__ uint32_t max_s16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.s16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t min_s16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("min.s16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Four codes (features k .. k + 3 in va, vb) as the bytes of one word. fma(y, mult, 1.5 * 2^23)
+// rounds the exact product to the nearest integer, ties to even, into the low mantissa bits
+// (|y mult| < 2^22). CM 0: no clamp (absmax: the products already lie in [-Q, Q]); CM 1: clamp
+// to [-8, 7] on the 16-bit lanes that hold the integers, exact while each fits an int16; CM 2:
+// clamp the integer-valued sums themselves, exact always.
+template <int CM>
+__device__ __forceinline__ uint32_t codes4(float2 va, float2 vb, float2 mult2) {
+  const float2 magic2 = make_float2(12582912.f, 12582912.f);
+  float2 p0 = __ffma2_rn(va, mult2, magic2);
+  float2 p1 = __ffma2_rn(vb, mult2, magic2);
+  if constexpr (CM == 2) {
+    constexpr float lo = 12582912.f - 8.f, hi = 12582912.f + 7.f;
+    p0.x = fminf(fmaxf(p0.x, lo), hi);
+    p0.y = fminf(fmaxf(p0.y, lo), hi);
+    p1.x = fminf(fmaxf(p1.x, lo), hi);
+    p1.y = fminf(fmaxf(p1.y, lo), hi);
+  }
+  uint32_t h0 = __byte_perm(__float_as_uint(p0.x), __float_as_uint(p0.y), 0x5410);  // int16 lanes k, k+1
+  uint32_t h1 = __byte_perm(__float_as_uint(p1.x), __float_as_uint(p1.y), 0x5410);
+  if constexpr (CM == 1) {
+    h0 = min_s16x2(max_s16x2(h0, 0xfff8fff8u), 0x00070007u);
+    h1 = min_s16x2(max_s16x2(h1, 0xfff8fff8u), 0x00070007u);
+  }
+  return __byte_perm(h0, h1, 0x6420);
+}
+
+// The codes of one thread's 128 values: v[4m .. 4m + 3] are the 8 consecutive features
+// base + 64 m + 0..7. Each run is one store: lanes 8j .. 8j + 7 of a warp cover 64 (int8) or 32
+// (packed int4: low nibble = even feature) contiguous bytes.
+template <int CM>
+__device__ __forceinline__ void quant_store(const float2* v, float2 mult2, uint8_t* row_codes, bool packed4,
+                                            int base) {
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    const uint32_t w0 = codes4<CM>(v[4 * m], v[4 * m + 1], mult2);
+    const uint32_t w1 = codes4<CM>(v[4 * m + 2], v[4 * m + 3], mult2);
+    if (!packed4) {
+      *reinterpret_cast<uint2*>(row_codes + base + 64 * m) = make_uint2(w0, w1);
+    } else {
+      // byte 0 of z = code k | code k+1 << 4, byte 2 = code k+2 | code k+3 << 4 (bytes 1, 3 unused)
+      const uint32_t z0 = (w0 & 0x000f000fu) | ((w0 >> 4) & 0x00f000f0u);
+      const uint32_t z1 = (w1 & 0x000f000fu) | ((w1 >> 4) & 0x00f000f0u);
+      *reinterpret_cast<uint32_t*>(row_codes + base / 2 + 32 * m) = __byte_perm(z0, z1, 0x6420);
+    }
+  }
+}
+
 // QM: 0 = a8 absmax, 1 = a4 absmean, 2 = a4 absmax
 template <int QM>
-__global__ void __launch_bounds__(kNtThreads, 2) norm_fht_quant_tc_kernel(const NfqArgs a) {
+__global__ void __launch_bounds__(kNtThreads, kNtCtasPerSm) norm_fht_quant_tc_kernel(const NfqArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_nt[];
   __shared__ __align__(8) uint64_t land_full, land_empty, acc_full[2], acc_empty[2], drain_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
-  __shared__ float red_ss[4], red_st[4];
+  __shared__ float red_ss[2][4], red_st[2][4];  // by row parity: one barrier per row suffices
 
   constexpr int K = kNtN;
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_nt) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_shared<1024>(smem_nt);
   uint8_t* hA = smem;                 // H_128, two K halves of [128 rows][128 B], 128-byte swizzle
   uint8_t* land = smem + 32768;       // the bf16 row
-  uint8_t* cbuf = land + kNtRowBytes; // codes [k mod 8][k / 8]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nrows = a.M > (int)blockIdx.x ? (a.M - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
@@ -162,7 +236,7 @@ __global__ void __launch_bounds__(kNtThreads, 2) norm_fht_quant_tc_kernel(const 
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(as * 128);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)  // a' = 16 ks .. 16 ks + 15: k bits 13..10 = 2ks, 2ks+1
+        for (int ks = 0; ks < 8; ++ks)  // a' = 16 ks .. 16 ks + 15, a' bits 6..4 = ks = k bits 13..11
           mma_bf16(d, smem_desc_sw128(smem_u32(hA + (ks >> 2) * 16384 + (ks & 3) * 32)),
                    smem_desc_none(smem_u32(land + ks * 4096), 2048u, 128u), idesc, ks > 0 ? 1u : 0u);
         any = true;
@@ -191,11 +265,10 @@ __global__ void __launch_bounds__(kNtThreads, 2) norm_fht_quant_tc_kernel(const 
       }
     }
   } else {
-    // ---------------- consumers: thread = accumulator row a (k bits 13..10 = a >> 3, 2..0 = a & 7)
+    // ---------------- consumers: thread = accumulator row a (a bits 2..0 = k bits 5..3, a bits 6..3 =
+    // k bits 13..10)
     const int arow = warp * 32 + lane;
-    const int lo3 = arow & 7, hi4 = arow >> 3;
     constexpr float kQ = QM == 0 ? 127.f : (QM == 1 ? 2.6457513110645906f : 7.f);
-    constexpr int kLo = QM == 0 ? -128 : -8, kHi = QM == 0 ? 127 : 7;
     constexpr bool kAbsmax = QM != 1;
     const bool packed4 = (a.fmt == 0) && (QM != 0);
     for (int i = 0; i < nrows; ++i) {
@@ -248,13 +321,14 @@ __global__ void __launch_bounds__(kNtThreads, 2) norm_fht_quant_tc_kernel(const 
         st = kAbsmax ? fmaxf(st, t) : st + t;
       }
       if (lane == 0) {
-        red_ss[warp] = ss;
-        red_st[warp] = st;
+        red_ss[as][warp] = ss;
+        red_st[as][warp] = st;
       }
       consumer_bar();
-      ss = (red_ss[0] + red_ss[1]) + (red_ss[2] + red_ss[3]);  // fixed order, the same in every thread
-      st = kAbsmax ? fmaxf(fmaxf(red_st[0], red_st[1]), fmaxf(red_st[2], red_st[3]))
-                   : (red_st[0] + red_st[1]) + (red_st[2] + red_st[3]);
+      const float* rs_ = red_ss[as];
+      const float* rt_ = red_st[as];
+      ss = (rs_[0] + rs_[1]) + (rs_[2] + rs_[3]);  // fixed order, the same in every thread
+      st = kAbsmax ? fmaxf(fmaxf(rt_[0], rt_[1]), fmaxf(rt_[2], rt_[3])) : (rt_[0] + rt_[1]) + (rt_[2] + rt_[3]);
 
       // ---- per-row multiplier and scale (y = the unnormalised transform of x)
       const float r_rms = sqrtf(ss / (128.f * (float)K) + a.eps_norm);
@@ -271,74 +345,21 @@ __global__ void __launch_bounds__(kNtThreads, 2) norm_fht_quant_tc_kernel(const 
       }
       if (arow == 0) a.s_x[row] = sx;
 
-      // ---- codes of k = hi4 * 1024 + 8 n + lo3 for n = 0..127: row lo3, columns hi4*128 + n of
-      // the [k mod 8][k / 8] byte matrix; fp32 product, clamp (absmean), round by the 1.5 * 2^23 add
+      // ---- codes. Register pair v[4m + q] holds n = 8m + 2q and 8m + 2q + 1, so v[4m .. 4m + 3]
+      // are the 8 consecutive features k = base + 64 m + 0..7, base = 8 (a & 7) + 1024 (a >> 3).
+      // The absmean clamp runs on 16-bit lanes when every rounded product fits an int16: |y mult|
+      // <= mult ||y||_2 and ||y||_2^2 = 128 ss, so mult sqrt(128 ss) < 30000 guarantees it with room
+      // for fp32 rounding. The choice is the same in every consumer thread.
       const float2 mult2 = make_float2(mult, mult);
-      const float2 magic2 = make_float2(12582912.f, 12582912.f);
-      uint8_t* dst = cbuf + lo3 * kNtCrow + hi4 * 128;
-#pragma unroll
-      for (int j = 0; j < 128; j += 16) {
-        uint32_t wds[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int r0 = j + 4 * q;
-          float2 t0 = __fmul2_rn(v[r0 / 2], mult2);
-          float2 t1 = __fmul2_rn(v[r0 / 2 + 1], mult2);
-          if constexpr (!kAbsmax) {
-            t0.x = fminf(fmaxf(t0.x, (float)kLo), (float)kHi);
-            t0.y = fminf(fmaxf(t0.y, (float)kLo), (float)kHi);
-            t1.x = fminf(fmaxf(t1.x, (float)kLo), (float)kHi);
-            t1.y = fminf(fmaxf(t1.y, (float)kLo), (float)kHi);
-          }
-          const float2 p0 = __fadd2_rn(t0, magic2);
-          const float2 p1 = __fadd2_rn(t1, magic2);
-          const uint32_t h0 = __byte_perm(__float_as_uint(p0.x), __float_as_uint(p0.y), 0x5410);
-          const uint32_t h1 = __byte_perm(__float_as_uint(p1.x), __float_as_uint(p1.y), 0x5410);
-          wds[q] = __byte_perm(h0, h1, 0x6420);
-        }
-        *reinterpret_cast<uint4*>(dst + j) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+      const int base = (arow & 7) * 8 + (arow >> 3) * 1024;
+      uint8_t* row_codes = a.codes + (size_t)row * (packed4 ? K / 2 : K);
+      if constexpr (kAbsmax) {
+        quant_store<0>(v, mult2, row_codes, packed4, base);
+      } else if (mult * sqrtf(128.f * ss) < 30000.f) {
+        quant_store<1>(v, mult2, row_codes, packed4, base);
+      } else {
+        quant_store<2>(v, mult2, row_codes, packed4, base);
       }
-      consumer_bar();
-
-      // ---- stream the codes out in natural order, 32 consecutive codes per unit
-#pragma unroll
-      for (int it = 0; it < (K / 32) / 128; ++it) {
-        const int vcol = arow + it * 128;
-        const uint8_t* srcc = cbuf + 4 * vcol;
-        uint32_t w[8];
-#pragma unroll
-        for (int b = 0; b < 8; ++b) w[b] = *reinterpret_cast<const uint32_t*>(srcc + b * kNtCrow);
-        // byte j of w[b] is the code of k = 32 * vcol + 8 * j + b
-        if (!packed4) {
-          uint32_t o[8];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t a01l = __byte_perm(w[4 * h], w[4 * h + 1], 0x5140);
-            const uint32_t a01h = __byte_perm(w[4 * h], w[4 * h + 1], 0x7362);
-            const uint32_t a23l = __byte_perm(w[4 * h + 2], w[4 * h + 3], 0x5140);
-            const uint32_t a23h = __byte_perm(w[4 * h + 2], w[4 * h + 3], 0x7362);
-            o[0 + h] = __byte_perm(a01l, a23l, 0x5410);
-            o[2 + h] = __byte_perm(a01l, a23l, 0x7632);
-            o[4 + h] = __byte_perm(a01h, a23h, 0x5410);
-            o[6 + h] = __byte_perm(a01h, a23h, 0x7632);
-          }
-          uint4* dstg = reinterpret_cast<uint4*>(a.codes + (size_t)row * K + 32 * vcol);
-          dstg[0] = make_uint4(o[0], o[1], o[2], o[3]);
-          dstg[1] = make_uint4(o[4], o[5], o[6], o[7]);
-        } else {
-          uint32_t m[4];
-#pragma unroll
-          for (int i2 = 0; i2 < 4; ++i2) m[i2] = (w[2 * i2] & 0x0f0f0f0fu) | ((w[2 * i2 + 1] & 0x0f0f0f0fu) << 4);
-          const uint32_t a01l = __byte_perm(m[0], m[1], 0x5140);
-          const uint32_t a01h = __byte_perm(m[0], m[1], 0x7362);
-          const uint32_t a23l = __byte_perm(m[2], m[3], 0x5140);
-          const uint32_t a23h = __byte_perm(m[2], m[3], 0x7362);
-          const uint4 o = make_uint4(__byte_perm(a01l, a23l, 0x5410), __byte_perm(a01l, a23l, 0x7632),
-                                     __byte_perm(a01h, a23h, 0x5410), __byte_perm(a01h, a23h, 0x7632));
-          *reinterpret_cast<uint4*>(a.codes + (size_t)row * (K / 2) + 16 * vcol) = o;
-        }
-      }
-      // the next row's statistics barrier orders these reads before the matrix is rewritten
     }
   }
   tc_fence_before();

@@ -33,9 +33,10 @@ Readings taken where the pages are silent or the formulas were dropped
        a4 absmax : gamma = max|x|, q = RoundClip(7 x/(gamma+eps), -8, 7),    s = gamma/7
      A row whose statistic is zero (and eps = 0) gives q = 0 and s = 0.
   R5 RoundClip rounds to nearest, ties to even. The rounding decision is taken
-     on float32 operands in float32 (the precision the GPU kernel decides in):
-     the element and the per-row multiplier are rounded to float32, multiplied
-     in float32, then rounded to an integer. Everything before that is float64.
+     on float32 operands: the element and the per-row multiplier are rounded to
+     float32 and their exact product (which float64 holds without error) is
+     rounded once to an integer, as a fused multiply-add does on the GPU.
+     Everything before that is float64.
   R6 output: y[m, n] = s[m] * alpha * sum_k q[m, k] t[k, n], evaluated in float64.
 
 Parity status: the transform, the quantisers, the ternariser and the integer
@@ -152,8 +153,8 @@ def hadamard_transform(x: np.ndarray, block: int = 0) -> np.ndarray:
 
 
 def _round_clip_f32(x: np.ndarray, mult: np.ndarray, lo: int, hi: int) -> np.ndarray:
-    """RoundClip with the decision taken in float32 (reading R5)."""
-    v = x.astype(np.float32) * mult.astype(np.float32)  # float32 product of float32 operands
+    """RoundClip on float32 operands (reading R5): the exact product, rounded once."""
+    v = x.astype(np.float32).astype(np.float64) * mult.astype(np.float32).astype(np.float64)  # 24 x 24 bits: exact
     return np.clip(np.rint(v), lo, hi).astype(np.int8)  # ties to even
 
 

@@ -100,8 +100,11 @@ def test_norm_fht_quant_matches_oracle(K, had_block, M, quant, fmt, use_gain):
     np.testing.assert_allclose(s, s_ref, rtol=1e-5)
 
 
-def test_norm_fht_quant_degenerate_rows():
-    K = 2048
+@pytest.mark.parametrize("K,fmt", [(2048, hbl.HBL_CODES_I8), (16384, hbl.HBL_CODES_I8),
+                                   (16384, hbl.HBL_CODES_PACKED)])
+def test_norm_fht_quant_degenerate_rows(K, fmt):
+    # at K = 16384 the constant row's transform is one spike of sqrt(7) K > 2^15 codes before
+    # clamping: the 16384-wide kernel must take its clamp for rounded values outside int16
     x = np.zeros((6, K), dtype=np.float32)
     x[1, 5] = 3.0                      # single spike: transform is flat, all |codes| equal
     x[2] = -1.0                        # constant row: transform is a single spike
@@ -112,7 +115,7 @@ def test_norm_fht_quant_degenerate_rows():
     for quant in QUANT_NAME:
         abits, mode = QUANT_NAME[quant]
         q_ref, s_ref = oracle.norm_fht_quant(bits, None, 0, abits, mode)
-        q, s = gpu_codes(bits, None, 0, quant, hbl.HBL_CODES_I8)
+        q, s = gpu_codes(bits, None, 0, quant, fmt)
         assert_codes_close(q, q_ref)
         assert np.all(q[0] == 0) and s[0] == 0.0
         np.testing.assert_allclose(s[1:], s_ref[1:], rtol=1e-5)

@@ -128,17 +128,28 @@ def test_quantiser_defining_properties(abits, mode, Q, lo, hi):
         np.testing.assert_array_equal(np.abs(q[np.arange(64), am]), int(Q))
 
 
+def test_rounding_takes_the_exact_product():
+    # x = 1 + 2^-23 and mult = 2.5 - 2^-22 are float32 values whose exact product is
+    # 2.5 + 2^-24 - 2^-45: just above the tie, so the code is 3. Rounding the product to float32
+    # first would land exactly on 2.5 and give the even code 2.
+    x = np.array([1.0 + 2.0 ** -23])
+    mult = np.array([2.5 - 2.0 ** -22])
+    assert np.float32(x[0]) == x[0] and np.float32(mult[0]) == mult[0]
+    assert float(np.float32(x[0]) * np.float32(mult[0])) == 2.5
+    assert oracle.hbl_oracle._round_clip_f32(x, mult, -8, 7)[0] == 3
+
+
 @pytest.mark.parametrize("abits,mode,Q,lo,hi", QUANTS)
 def test_quantiser_brute_force_nearest_code(abits, mode, Q, lo, hi):
-    # brute force: among all codes in [lo, hi] the oracle picks the one nearest to the
-    # float32 value it decides on (ties to the even code).
+    # brute force: among all codes in [lo, hi] the oracle picks the one nearest to the exact
+    # product of the float32 element and the float32 multiplier (ties to the even code).
     x = RNG.standard_normal((8, 32))
     q, s = oracle.quantize(x, abits, mode)
     stat = np.abs(x).max(axis=1) if mode == "absmax" else np.abs(x).mean(axis=1)
     for m in range(8):
         mult = np.float32(Q / stat[m])
         for k in range(32):
-            vv = float(np.float32(x[m, k]) * mult)
+            vv = float(np.float32(x[m, k])) * float(mult)  # exact in a Python float
             best = min(range(lo, hi + 1), key=lambda c: (abs(vv - c), c % 2))
             assert q[m, k] == best, (m, k, vv, q[m, k], best)
 
