@@ -41,7 +41,7 @@ WORKLOAD = ("7B-like H-BitLinear layer pair: Wo 4096->4096 + Wdown 16384->4096, 
 # source it was taken on (reported as null once the source has changed).
 NCU_TRAFFIC = {
     # profiles/gemm_tc2_wdown_7b_m8192.md: dram__bytes_read.sum + dram__bytes_write.sum
-    "gemm_tc2[wdown_7b_a4]": {"bytes": 611.340544e6 + 73.249024e6, "src": "gemm_tc2.cuh", "sha": "8eab555aa3d677d4"},
+    "gemm_tc2[wdown_7b_a4]": {"bytes": 600.112896e6 + 69.806592e6, "src": "gemm_tc2.cuh", "sha": "2cc3da467c32c2e2"},
 }
 
 
@@ -54,7 +54,7 @@ def product_kernel(M):
 
 def nfq_kernel(K, had_block):
     """Name of the fused activation kernel hbl_norm_fht_quant runs (no gain)."""
-    return "norm_fht_quant_tc" if (K == 16384 and had_block == 0) else "norm_fht_quant"
+    return "norm_fht_quant_tc" if (K in (8192, 16384) and had_block == 0) else "norm_fht_quant"
 
 
 def weight_bytes(M, K, N):
@@ -477,6 +477,58 @@ def run_profile_product(M):
     print(f"product {product_kernel(M)[0]}: M={M} K={spec.K} N={spec.N}, 3 launches", flush=True)
 
 
+ACTIVATION_CASES = [("wo_7b_a4", 8192), ("wdown_7b_a4", 8192), ("wdown_3b_a4", 4096),
+                    ("wdown_nonpow2_a4", 8192), ("wo_1p3b_a4", 2048)]
+
+
+def run_activation_only(reps=50):
+    """Times the fused activation kernel (hbl_norm_fht_quant, a4 absmean, int8 codes) alone on
+    each workload width, with CUDA events on its stream. Each launch works on the next of several
+    input/output copies whose total exceeds L2, so that no launch finds its data in L2. Prints one
+    line per workload (algorithmic bytes: the bf16 input, one code byte per feature, one scale per
+    row); no bench line."""
+    import torch
+
+    import hadamard_bit_quant_hbl_b200 as hbl
+
+    torch.cuda.set_device(0)
+    peak, _, _, peak_src = peaks()
+    for name, M in ACTIVATION_CASES:
+        spec = inputs.WORKLOADS[name].with_m(M)
+        K = spec.K
+        nbytes = M * K * 3 + M * 4
+        ncopy = max(2, -(-400_000_000 // nbytes))
+        X0 = torch.from_numpy(inputs.activations(spec).view(np.int16)).cuda().view(torch.bfloat16)
+        bufs = [(X0.clone(), torch.empty((M, K), dtype=torch.uint8, device="cuda"),
+                 torch.empty(M, dtype=torch.float32, device="cuda")) for _ in range(ncopy)]
+        del X0
+        s = torch.cuda.Stream()
+
+        def launch(j):
+            X, codes, sx = bufs[j % ncopy]
+            hbl.hbl_norm_fht_quant(X, None, spec.had_block, hbl.HBL_Q_A4_ABSMEAN, 1e-6, 0.0, hbl.HBL_CODES_I8,
+                                   codes, sx, stream=s.cuda_stream)
+
+        with torch.cuda.stream(s):
+            for j in range(max(5, ncopy)):
+                launch(j)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            for j in range(reps):
+                launch(j)
+            e1.record(s)
+        e1.synchronize()
+        st = hbl.hbl_device_status()
+        if st != hbl.HBL_OK:
+            raise RuntimeError(hbl.hbl_status_string(st))
+        us = e0.elapsed_time(e1) / reps * 1000
+        kern = nfq_kernel(K, spec.had_block)
+        print(f"{kern:18s} {name:18s} M={M:5d} K={K:6d} had_block={spec.had_block:4d} {us:8.1f} us "
+              f"{nbytes / us / 1e3:7.1f} GB/s {nbytes / us / 1e3 / peak:6.3f} of {peak_src} HBM "
+              f"({ncopy} copies rotated)", flush=True)
+        del bufs
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -491,7 +543,12 @@ def main():
     ap.add_argument("--sweep-steps", type=int, default=100)
     ap.add_argument("--profile-product", type=int, default=0, metavar="M",
                     help="only run the Wdown product three times with M tokens (an ncu target); no bench line")
+    ap.add_argument("--activation-only", action="store_true",
+                    help="only time the fused activation kernel alone on each workload width; no bench line")
     args = ap.parse_args()
+    if args.activation_only:
+        run_activation_only()
+        return
     if args.profile_product:
         run_profile_product(args.profile_product)
         return

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "hbl.h"
 
@@ -150,18 +151,20 @@ constexpr int eb_for(int L) {
   return L == 8 ? 4 : L == 9 ? 5 : L == 10 ? 5 : L == 11 ? 6 : L == 12 ? 6 : 7;
 }
 
-// The 16384-wide transform with the H_128 factor on the tensor cores (no gain, one block).
-template <int QM>
+// Transforms of 2^L features (one block, no gain) with the H_128 factor on the tensor cores; the
+// grid walks groups of 2^(14-L) rows, two CTAs per SM.
+template <int QM, int L>
 hbl_status launch_nfq_tc(const NfqArgs& a, cudaStream_t s) {
   static SmemLimit lim;
-  auto* k = norm_fht_quant_tc_kernel<QM>;
+  auto* k = norm_fht_quant_tc_kernel<QM, L>;
   cudaError_t e = allow_smem(k, kNtSmem, lim);
   if (e != cudaSuccess) return cuda_fail(e);
   cudaLaunchConfig_t cfg = {};
   int dev = 0;
   cudaGetDevice(&dev);
   const int resident = kNtCtasPerSm * device_sms(dev);
-  cfg.gridDim = dim3(a.M < resident ? a.M : resident, 1, 1);
+  const int groups = (a.M + (kNtN >> L) - 1) / (kNtN >> L);  // 2^(14-L) rows per group
+  cfg.gridDim = dim3(groups < resident ? groups : resident, 1, 1);
   cfg.blockDim = dim3(kNtThreads, 1, 1);
   cfg.dynamicSmemBytes = kNtSmem;
   cfg.stream = s;
@@ -221,10 +224,18 @@ hbl_status run_nfq(const void* X, const float* gain, int M, int K, int had_block
   a.groups = (M + rows - 1) / rows;
   a.pf_dist = 0;
 
-  if (L == 14 && nb == 1 && gain == nullptr) {
-    if (quant == 0) return launch_nfq_tc<0>(a, stream);
-    if (quant == 1) return launch_nfq_tc<1>(a, stream);
-    return launch_nfq_tc<2>(a, stream);
+  // One block of 2^13 or 2^14 features, no gain: the tensor-core kernel. (It also serves 2^11 and
+  // 2^12, correctly, but measured slower there than the CUDA-core kernel: with 8 and 4 rows per
+  // group the per-row statistics and scalars outweigh the butterflies it saves.)
+  if ((L == 13 || L == 14) && nb == 1 && gain == nullptr) {
+    auto tc = [&](auto lc) -> hbl_status {
+      constexpr int LL = decltype(lc)::value;
+      if (quant == 0) return launch_nfq_tc<0, LL>(a, stream);
+      if (quant == 1) return launch_nfq_tc<1, LL>(a, stream);
+      return launch_nfq_tc<2, LL>(a, stream);
+    };
+    if (L == 13) return tc(std::integral_constant<int, 13>{});
+    return tc(std::integral_constant<int, 14>{});
   }
   // K <= 32768 bounds nb, so these R always suffice: L=8 nb<=128 (R<=4), L=9..12 R<=2, L>=13 R=1
   switch (L) {

@@ -144,43 +144,49 @@ __device__ __forceinline__ uint32_t codes4(float2 va, float2 vb, float2 mult2) {
   return __byte_perm(h0, h1, 0x6420);
 }
 
-// The codes of one thread's 128 values: v[4m .. 4m + 3] are the 8 consecutive features
-// base + 64 m + 0..7. Each run is one store: lanes 8j .. 8j + 7 of a warp cover 64 (int8) or 32
-// (packed int4: low nibble = even feature) contiguous bytes.
-template <int CM>
+// The codes of one row's runs in one thread: v[4u .. 4u + 3] are the 8 consecutive features
+// 8a + 1024u + 0..7 of the row (a = the thread's accumulator lane). Each run is one store, and the
+// 32 lanes of a warp (consecutive a) cover 256 (int8) or 128 (packed int4, low nibble = even
+// feature) contiguous bytes.
+template <int CM, int RUNS>
 __device__ __forceinline__ void quant_store(const float2* v, float2 mult2, uint8_t* row_codes, bool packed4,
-                                            int base) {
+                                            int a) {
 #pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    const uint32_t w0 = codes4<CM>(v[4 * m], v[4 * m + 1], mult2);
-    const uint32_t w1 = codes4<CM>(v[4 * m + 2], v[4 * m + 3], mult2);
+  for (int u = 0; u < RUNS; ++u) {
+    const uint32_t w0 = codes4<CM>(v[4 * u], v[4 * u + 1], mult2);
+    const uint32_t w1 = codes4<CM>(v[4 * u + 2], v[4 * u + 3], mult2);
     if (!packed4) {
-      *reinterpret_cast<uint2*>(row_codes + base + 64 * m) = make_uint2(w0, w1);
+      *reinterpret_cast<uint2*>(row_codes + 8 * a + 1024 * u) = make_uint2(w0, w1);
     } else {
       // byte 0 of z = code k | code k+1 << 4, byte 2 = code k+2 | code k+3 << 4 (bytes 1, 3 unused)
       const uint32_t z0 = (w0 & 0x000f000fu) | ((w0 >> 4) & 0x00f000f0u);
       const uint32_t z1 = (w1 & 0x000f000fu) | ((w1 >> 4) & 0x00f000f0u);
-      *reinterpret_cast<uint32_t*>(row_codes + base / 2 + 32 * m) = __byte_perm(z0, z1, 0x6420);
+      *reinterpret_cast<uint32_t*>(row_codes + 4 * a + 512 * u) = __byte_perm(z0, z1, 0x6420);
     }
   }
 }
 
-// QM: 0 = a8 absmax, 1 = a4 absmean, 2 = a4 absmax
-template <int QM>
+// QM: 0 = a8 absmax, 1 = a4 absmean, 2 = a4 absmax. L: log2 K, 11..14; a group of 2^(14-L) rows.
+template <int QM, int L>
 __global__ void __launch_bounds__(kNtThreads, kNtCtasPerSm) norm_fht_quant_tc_kernel(const NfqArgs a) {
+  static_assert(L >= 11 && L <= 14, "the group must fill 16384 elements with at most 8 rows");
+  constexpr int K = 1 << L;
+  constexpr int R = kNtN / K;   // rows per group
+  constexpr int NB = K / 128;   // accumulator columns (values of n) per row
+  constexpr int RUNS = NB / 8;  // runs of 8 consecutive features per row and thread
   extern __shared__ __align__(1024) uint8_t smem_nt[];
   __shared__ __align__(8) uint64_t land_full, land_empty, acc_full[2], acc_empty[2], drain_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
-  __shared__ float red_ss[2][4], red_st[2][4];  // by row parity: one barrier per row suffices
+  __shared__ float red_ss[2][R][4], red_st[2][R][4];  // by group parity: one barrier per group suffices
 
-  constexpr int K = kNtN;
   uint8_t* smem = align_shared<1024>(smem_nt);
   uint8_t* hA = smem;                 // H_128, two K halves of [128 rows][128 B], 128-byte swizzle
-  uint8_t* land = smem + 32768;       // the bf16 row
+  uint8_t* land = smem + 32768;       // the group's R bf16 rows, 16384 elements
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nrows = a.M > (int)blockIdx.x ? (a.M - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+  const int ngroups = (a.M + R - 1) / R;
+  const int ng = ngroups > (int)blockIdx.x ? (ngroups - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
 
   // X (and the codes buffer) may belong to the kernel before this one: wait for it
   pdl_wait();
@@ -219,34 +225,39 @@ __global__ void __launch_bounds__(kNtThreads, kNtCtasPerSm) norm_fht_quant_tc_ke
   const uint32_t tmem_base = tmem_slot;
 
   if (warp == 4) {
-    // ---------------- row copies and MMAs (one thread)
+    // ---------------- group copies and MMAs (one thread)
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(128, 128);
+      // the rows of group g that exist, as one contiguous copy (a ragged last group copies fewer;
+      // the columns of the missing rows then hold stale values that nothing stores)
+      auto copy_group = [&](int g) {
+        const int rows = a.M - g * R < R ? a.M - g * R : R;
+        const uint32_t bytes = (uint32_t)rows * (uint32_t)K * 2u;
+        mbar_arrive_expect_tx(&land_full, bytes);
+        bulk_load_1d(land, a.X + (size_t)g * R * K, bytes, &land_full);
+      };
       int issued = 0;
       bool ok = true, any = false;
-      if (nrows > 0) {
-        mbar_arrive_expect_tx(&land_full, (uint32_t)kNtRowBytes);
-        bulk_load_1d(land, a.X + (size_t)blockIdx.x * K, (uint32_t)kNtRowBytes, &land_full);
+      if (ng > 0) {
+        copy_group((int)blockIdx.x);
         issued = 1;
       }
-      for (int i = 0; i < nrows; ++i) {
+      for (int i = 0; i < ng; ++i) {
         const int as = i & 1;
         if (!mbar_wait(&land_full, (uint32_t)i & 1u, &abort_flag)) { ok = false; break; }
         if (!mbar_wait(&acc_empty[as], ((uint32_t)(i >> 1) & 1u) ^ 1u, &abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(as * 128);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)  // a' = 16 ks .. 16 ks + 15, a' bits 6..4 = ks = k bits 13..11
+        for (int ks = 0; ks < 8; ++ks)  // a' = 16 ks .. 16 ks + 15, a' bits 6..4 = ks = k bits 9..7
           mma_bf16(d, smem_desc_sw128(smem_u32(hA + (ks >> 2) * 16384 + (ks & 3) * 32)),
-                   smem_desc_none(smem_u32(land + ks * 4096), 2048u, 128u), idesc, ks > 0 ? 1u : 0u);
+                   smem_desc_none(smem_u32(land + ks * 256), 128u, 2048u), idesc, ks > 0 ? 1u : 0u);
         any = true;
         mma_commit(&acc_full[as]);
         mma_commit(&land_empty);
-        if (issued < nrows) {  // the next row, once the MMAs have read this one
+        if (issued < ng) {  // the next group, once the MMAs have read this one
           if (!mbar_wait(&land_empty, (uint32_t)i & 1u, &abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&land_full, (uint32_t)kNtRowBytes);
-          bulk_load_1d(land, a.X + ((size_t)blockIdx.x + (size_t)issued * gridDim.x) * K, (uint32_t)kNtRowBytes,
-                       &land_full);
+          copy_group((int)blockIdx.x + issued * (int)gridDim.x);
           ++issued;
         }
       }
@@ -265,20 +276,21 @@ __global__ void __launch_bounds__(kNtThreads, kNtCtasPerSm) norm_fht_quant_tc_ke
       }
     }
   } else {
-    // ---------------- consumers: thread = accumulator row a (a bits 2..0 = k bits 5..3, a bits 6..3 =
-    // k bits 13..10)
+    // ---------------- consumers: thread = accumulator lane a = k bits 9..3 of every row
     const int arow = warp * 32 + lane;
     constexpr float kQ = QM == 0 ? 127.f : (QM == 1 ? 2.6457513110645906f : 7.f);
     constexpr bool kAbsmax = QM != 1;
+    constexpr int PER = R >= 4 ? 1 : 4 / R;  // independent accumulators per row
     const bool packed4 = (a.fmt == 0) && (QM != 0);
-    for (int i = 0; i < nrows; ++i) {
+    for (int i = 0; i < ng; ++i) {
       const int as = i & 1;
-      const int row = (int)blockIdx.x + i * (int)gridDim.x;
+      const int g = (int)blockIdx.x + i * (int)gridDim.x;
       const bool got = mbar_wait(&acc_full[as], (uint32_t)(i >> 1) & 1u, &abort_flag);
       if (consumer_bar_or(!got || abort_flag)) break;  // the same decision in every consumer
       tc_fence_after();
 
-      // ---- the 128 columns of this lane: D[a][n], n = k bits 9..3
+      // ---- the 128 columns of this lane: column r NB + 8 nh + nl is D[a] of row r at the features
+      // 1024 nh + 8 a + nl
       float2 v[64];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -289,76 +301,121 @@ __global__ void __launch_bounds__(kNtThreads, kNtCtasPerSm) norm_fht_quant_tc_ke
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[as]);  // the accumulator may take the row after next
+      if (lane == 0) mbar_arrive(&acc_empty[as]);  // the accumulator may take the group after next
 
-      // sum of squares: sum_a,n D^2 = 128 sum x^2 (H_128 has orthogonal rows of norm^2 128)
-      float2 ss2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      // sum of squares per row: sum_a,n D^2 = 128 sum x^2 (H_128 has orthogonal rows of norm^2 128)
+      float ss[R], st[R];
+      {
+        float2 acc[R * PER];
 #pragma unroll
-      for (int j = 0; j < 64; ++j) ss2[j & 3] = __ffma2_rn(v[j], v[j], ss2[j & 3]);
-      float ss = ((ss2[0].x + ss2[0].y) + (ss2[1].x + ss2[1].y)) + ((ss2[2].x + ss2[2].y) + (ss2[3].x + ss2[3].y));
-
-      fwht_regs2<128, 7>(v);  // the factor over n
-
-      float st;
-      if constexpr (kAbsmax) {
-        float sta[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int q = 0; q < R * PER; ++q) acc[q] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int j = 0; j < 64; ++j) sta[j & 3] = fmaxf(sta[j & 3], fmaxf(fabsf(v[j].x), fabsf(v[j].y)));
-        st = fmaxf(fmaxf(sta[0], sta[1]), fmaxf(sta[2], sta[3]));
-      } else {
-        float2 sta2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-        for (int j = 0; j < 64; j += 2) {
-          const float2 t = make_float2(fabsf(v[j].x) + fabsf(v[j].y), fabsf(v[j + 1].x) + fabsf(v[j + 1].y));
-          sta2[(j / 2) & 3] = __fadd2_rn(sta2[(j / 2) & 3], t);
+        for (int j = 0; j < 64; ++j) {
+          const int q = (2 * j / NB) * PER + (j % PER);
+          acc[q] = __ffma2_rn(v[j], v[j], acc[q]);
         }
-        st = ((sta2[0].x + sta2[0].y) + (sta2[1].x + sta2[1].y)) + ((sta2[2].x + sta2[2].y) + (sta2[3].x + sta2[3].y));
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          float t = 0.f;
+#pragma unroll
+          for (int q = 0; q < PER; ++q) t += acc[r * PER + q].x + acc[r * PER + q].y;
+          ss[r] = t;
+        }
+      }
+
+      fwht_regs2<128, L - 7>(v);  // the factor over n, within each row
+
+      if constexpr (kAbsmax) {
+        float acc[R * PER];
+#pragma unroll
+        for (int q = 0; q < R * PER; ++q) acc[q] = 0.f;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const int q = (2 * j / NB) * PER + (j % PER);
+          acc[q] = fmaxf(acc[q], fmaxf(fabsf(v[j].x), fabsf(v[j].y)));
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          float t = 0.f;
+#pragma unroll
+          for (int q = 0; q < PER; ++q) t = fmaxf(t, acc[r * PER + q]);
+          st[r] = t;
+        }
+      } else {
+        float2 acc[R * PER];
+#pragma unroll
+        for (int q = 0; q < R * PER; ++q) acc[q] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < 64; j += 2) {  // v[j], v[j + 1]: the same row
+          const int q = (2 * j / NB) * PER + ((j / 2) % PER);
+          const float2 t = make_float2(fabsf(v[j].x) + fabsf(v[j].y), fabsf(v[j + 1].x) + fabsf(v[j + 1].y));
+          acc[q] = __fadd2_rn(acc[q], t);
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          float t = 0.f;
+#pragma unroll
+          for (int q = 0; q < PER; ++q) t += acc[r * PER + q].x + acc[r * PER + q].y;
+          st[r] = t;
+        }
       }
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) {
-        ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        const float t = __shfl_xor_sync(0xffffffffu, st, o);
-        st = kAbsmax ? fmaxf(st, t) : st + t;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          ss[r] += __shfl_xor_sync(0xffffffffu, ss[r], o);
+          const float t = __shfl_xor_sync(0xffffffffu, st[r], o);
+          st[r] = kAbsmax ? fmaxf(st[r], t) : st[r] + t;
+        }
       }
       if (lane == 0) {
-        red_ss[as][warp] = ss;
-        red_st[as][warp] = st;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          red_ss[as][r][warp] = ss[r];
+          red_st[as][r][warp] = st[r];
+        }
       }
       consumer_bar();
-      const float* rs_ = red_ss[as];
-      const float* rt_ = red_st[as];
-      ss = (rs_[0] + rs_[1]) + (rs_[2] + rs_[3]);  // fixed order, the same in every thread
-      st = kAbsmax ? fmaxf(fmaxf(rt_[0], rt_[1]), fmaxf(rt_[2], rt_[3])) : (rt_[0] + rt_[1]) + (rt_[2] + rt_[3]);
 
-      // ---- per-row multiplier and scale (y = the unnormalised transform of x)
-      const float r_rms = sqrtf(ss / (128.f * (float)K) + a.eps_norm);
-      const float rs = r_rms * sqrtf((float)K);
-      const float sy = kAbsmax ? st : st / (float)K;
-      float mult, sx;
-      if (a.eps_q == 0.f) {
-        mult = sy > 0.f ? kQ / sy : 0.f;
-        sx = sy > 0.f ? sy / (rs * kQ) : 0.f;
-      } else {
-        const float stat = sy / rs;
-        mult = kQ / ((stat + a.eps_q) * rs);
-        sx = stat / kQ;
-      }
-      if (arow == 0) a.s_x[row] = sx;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int row = g * R + r;
+        if (row >= a.M) break;  // the same in every thread
+        const float* rs_ = red_ss[as][r];
+        const float* rt_ = red_st[as][r];
+        const float ssr = (rs_[0] + rs_[1]) + (rs_[2] + rs_[3]);  // fixed order, the same in every thread
+        const float str = kAbsmax ? fmaxf(fmaxf(rt_[0], rt_[1]), fmaxf(rt_[2], rt_[3]))
+                                  : (rt_[0] + rt_[1]) + (rt_[2] + rt_[3]);
 
-      // ---- codes. Register pair v[4m + q] holds n = 8m + 2q and 8m + 2q + 1, so v[4m .. 4m + 3]
-      // are the 8 consecutive features k = base + 64 m + 0..7, base = 8 (a & 7) + 1024 (a >> 3).
-      // The absmean clamp runs on 16-bit lanes when every rounded product fits an int16: |y mult|
-      // <= mult ||y||_2 and ||y||_2^2 = 128 ss, so mult sqrt(128 ss) < 30000 guarantees it with room
-      // for fp32 rounding. The choice is the same in every consumer thread.
-      const float2 mult2 = make_float2(mult, mult);
-      const int base = (arow & 7) * 8 + (arow >> 3) * 1024;
-      uint8_t* row_codes = a.codes + (size_t)row * (packed4 ? K / 2 : K);
-      if constexpr (kAbsmax) {
-        quant_store<0>(v, mult2, row_codes, packed4, base);
-      } else if (mult * sqrtf(128.f * ss) < 30000.f) {
-        quant_store<1>(v, mult2, row_codes, packed4, base);
-      } else {
-        quant_store<2>(v, mult2, row_codes, packed4, base);
+        // ---- per-row multiplier and scale (y = the unnormalised transform of x)
+        const float r_rms = sqrtf(ssr / (128.f * (float)K) + a.eps_norm);
+        const float rs = r_rms * sqrtf((float)K);
+        const float sy = kAbsmax ? str : str / (float)K;
+        float mult, sx;
+        if (a.eps_q == 0.f) {
+          mult = sy > 0.f ? kQ / sy : 0.f;
+          sx = sy > 0.f ? sy / (rs * kQ) : 0.f;
+        } else {
+          const float stat = sy / rs;
+          mult = kQ / ((stat + a.eps_q) * rs);
+          sx = stat / kQ;
+        }
+        if (arow == r) a.s_x[row] = sx;
+
+        // ---- codes. The absmean clamp runs on 16-bit lanes when every rounded product fits an
+        // int16: |y mult| <= mult ||y||_2 and ||y||_2^2 = NB ssr (the n stages scale the sum of
+        // squares by NB), so mult sqrt(NB ssr) < 30000 guarantees it with room for fp32 rounding.
+        // The choice is the same in every consumer thread.
+        const float2 mult2 = make_float2(mult, mult);
+        const float2* vr = v + r * (NB / 2);
+        uint8_t* row_codes = a.codes + (size_t)row * (packed4 ? K / 2 : K);
+        if constexpr (kAbsmax) {
+          quant_store<0, RUNS>(vr, mult2, row_codes, packed4, arow);
+        } else if (mult * sqrtf((float)NB * ssr) < 30000.f) {
+          quant_store<1, RUNS>(vr, mult2, row_codes, packed4, arow);
+        } else {
+          quant_store<2, RUNS>(vr, mult2, row_codes, packed4, arow);
+        }
       }
     }
   }
