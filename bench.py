@@ -54,7 +54,7 @@ def product_kernel(M):
 
 def nfq_kernel(K, had_block):
     """Name of the fused activation kernel hbl_norm_fht_quant runs (no gain)."""
-    return "norm_fht_quant_tc" if (K in (8192, 16384) and had_block == 0) else "norm_fht_quant"
+    return "norm_fht_quant_tc" if (K in (4096, 8192, 16384) and had_block == 0) else "norm_fht_quant"
 
 
 def weight_bytes(M, K, N):

@@ -224,16 +224,17 @@ hbl_status run_nfq(const void* X, const float* gain, int M, int K, int had_block
   a.groups = (M + rows - 1) / rows;
   a.pf_dist = 0;
 
-  // One block of 2^13 or 2^14 features, no gain: the tensor-core kernel. (It also serves 2^11 and
-  // 2^12, correctly, but measured slower there than the CUDA-core kernel: with 8 and 4 rows per
-  // group the per-row statistics and scalars outweigh the butterflies it saves.)
-  if ((L == 13 || L == 14) && nb == 1 && gain == nullptr) {
+  // One block of 2^12 .. 2^14 features, no gain: the tensor-core kernel. (It also serves 2^11
+  // correctly; an earlier version of its per-row epilogue measured slower there than the CUDA-core
+  // kernel, 12.5 against 7.1 us on 2048 x 2048, so 2^11 stays on CUDA cores until measured again.)
+  if (L >= 12 && L <= 14 && nb == 1 && gain == nullptr) {
     auto tc = [&](auto lc) -> hbl_status {
       constexpr int LL = decltype(lc)::value;
       if (quant == 0) return launch_nfq_tc<0, LL>(a, stream);
       if (quant == 1) return launch_nfq_tc<1, LL>(a, stream);
       return launch_nfq_tc<2, LL>(a, stream);
     };
+    if (L == 12) return tc(std::integral_constant<int, 12>{});
     if (L == 13) return tc(std::integral_constant<int, 13>{});
     return tc(std::integral_constant<int, 14>{});
   }

@@ -192,6 +192,28 @@ __global__ void __launch_bounds__(kNtThreads, kNtCtasPerSm) norm_fht_quant_tc_ke
   pdl_wait();
   pdl_launch_dependents();
 
+  // the rows of group g that exist, as one contiguous copy (a ragged last group copies fewer; the
+  // columns of the missing rows then hold stale values that nothing stores)
+  auto copy_group = [&](int g) {
+    const int rows = a.M - g * R < R ? a.M - g * R : R;
+    const uint32_t bytes = (uint32_t)rows * (uint32_t)K * 2u;
+    mbar_arrive_expect_tx(&land_full, bytes);
+    bulk_load_1d(land, a.X + (size_t)g * R * K, bytes, &land_full);
+  };
+  // barriers first, then the first group's copy, which lands while every thread builds H
+  if (warp == 4 && lane == 0) {
+    abort_flag = 0;
+    mbar_init(&land_full, 1);
+    mbar_init(&land_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&acc_full[s], 1);
+      mbar_init(&acc_empty[s], 4);  // one lane of each consumer warp
+    }
+    mbar_init(&drain_bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (ng > 0) copy_group((int)blockIdx.x);
+  }
+
   // ---- H_128 in the A-operand layout: element (a, a') = (-1)^popcount(a & a') as bf16, a' in
   // two halves of 64; within a half, 16-byte chunk c of row a sits at chunk c ^ (a & 7)
   for (int e = tid; e < 128 * 64; e += kNtThreads) {  // two elements per 32-bit store
@@ -203,17 +225,6 @@ __global__ void __launch_bounds__(kNtThreads, kNtCtasPerSm) norm_fht_quant_tc_ke
         v0 | (v1 << 16);
   }
   fence_proxy_async_shared();  // generic-proxy writes -> visible to the tensor core
-  if (tid == 0) {
-    abort_flag = 0;
-    mbar_init(&land_full, 1);
-    mbar_init(&land_empty, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&acc_full[s], 1);
-      mbar_init(&acc_empty[s], 4);  // one lane of each consumer warp
-    }
-    mbar_init(&drain_bar, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
   if (warp == 4) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                  ::"r"(smem_u32(&tmem_slot)), "r"(kNtTmemCols) : "memory");
@@ -228,20 +239,8 @@ __global__ void __launch_bounds__(kNtThreads, kNtCtasPerSm) norm_fht_quant_tc_ke
     // ---------------- group copies and MMAs (one thread)
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(128, 128);
-      // the rows of group g that exist, as one contiguous copy (a ragged last group copies fewer;
-      // the columns of the missing rows then hold stale values that nothing stores)
-      auto copy_group = [&](int g) {
-        const int rows = a.M - g * R < R ? a.M - g * R : R;
-        const uint32_t bytes = (uint32_t)rows * (uint32_t)K * 2u;
-        mbar_arrive_expect_tx(&land_full, bytes);
-        bulk_load_1d(land, a.X + (size_t)g * R * K, bytes, &land_full);
-      };
-      int issued = 0;
+      int issued = ng > 0 ? 1 : 0;  // the first group's copy is in flight
       bool ok = true, any = false;
-      if (ng > 0) {
-        copy_group((int)blockIdx.x);
-        issued = 1;
-      }
       for (int i = 0; i < ng; ++i) {
         const int as = i & 1;
         if (!mbar_wait(&land_full, (uint32_t)i & 1u, &abort_flag)) { ok = false; break; }
@@ -377,41 +376,47 @@ __global__ void __launch_bounds__(kNtThreads, kNtCtasPerSm) norm_fht_quant_tc_ke
       }
       consumer_bar();
 
+      // ---- per-row multiplier and scale (y = the unnormalised transform of x): row r in lane r of
+      // every warp, from the same sums in the same order, so every thread gets the same values
+      float mult_l, sx_l;
+      int lanes16_l;
+      {
+        const int r = lane < R ? lane : 0;
+        const float* rs_ = red_ss[as][r];
+        const float* rt_ = red_st[as][r];
+        const float ssr = (rs_[0] + rs_[1]) + (rs_[2] + rs_[3]);
+        const float str = kAbsmax ? fmaxf(fmaxf(rt_[0], rt_[1]), fmaxf(rt_[2], rt_[3]))
+                                  : (rt_[0] + rt_[1]) + (rt_[2] + rt_[3]);
+        const float r_rms = sqrtf(ssr / (128.f * (float)K) + a.eps_norm);
+        const float rs = r_rms * sqrtf((float)K);
+        const float sy = kAbsmax ? str : str / (float)K;
+        if (a.eps_q == 0.f) {
+          mult_l = sy > 0.f ? kQ / sy : 0.f;
+          sx_l = sy > 0.f ? sy / (rs * kQ) : 0.f;
+        } else {
+          const float stat = sy / rs;
+          mult_l = kQ / ((stat + a.eps_q) * rs);
+          sx_l = stat / kQ;
+        }
+        // the absmean clamp may run on 16-bit lanes when every rounded product fits an int16:
+        // |y mult| <= mult ||y||_2 and ||y||_2^2 = NB ssr (the n stages scale the sum of squares by
+        // NB), so mult sqrt(NB ssr) < 30000 guarantees it with room for fp32 rounding
+        lanes16_l = mult_l * sqrtf((float)NB * ssr) < 30000.f ? 1 : 0;
+      }
+      if (warp == 0 && lane < R && g * R + lane < a.M) a.s_x[g * R + lane] = sx_l;
+
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         const int row = g * R + r;
         if (row >= a.M) break;  // the same in every thread
-        const float* rs_ = red_ss[as][r];
-        const float* rt_ = red_st[as][r];
-        const float ssr = (rs_[0] + rs_[1]) + (rs_[2] + rs_[3]);  // fixed order, the same in every thread
-        const float str = kAbsmax ? fmaxf(fmaxf(rt_[0], rt_[1]), fmaxf(rt_[2], rt_[3]))
-                                  : (rt_[0] + rt_[1]) + (rt_[2] + rt_[3]);
-
-        // ---- per-row multiplier and scale (y = the unnormalised transform of x)
-        const float r_rms = sqrtf(ssr / (128.f * (float)K) + a.eps_norm);
-        const float rs = r_rms * sqrtf((float)K);
-        const float sy = kAbsmax ? str : str / (float)K;
-        float mult, sx;
-        if (a.eps_q == 0.f) {
-          mult = sy > 0.f ? kQ / sy : 0.f;
-          sx = sy > 0.f ? sy / (rs * kQ) : 0.f;
-        } else {
-          const float stat = sy / rs;
-          mult = kQ / ((stat + a.eps_q) * rs);
-          sx = stat / kQ;
-        }
-        if (arow == r) a.s_x[row] = sx;
-
-        // ---- codes. The absmean clamp runs on 16-bit lanes when every rounded product fits an
-        // int16: |y mult| <= mult ||y||_2 and ||y||_2^2 = NB ssr (the n stages scale the sum of
-        // squares by NB), so mult sqrt(NB ssr) < 30000 guarantees it with room for fp32 rounding.
-        // The choice is the same in every consumer thread.
+        const float mult = __shfl_sync(0xffffffffu, mult_l, r);
+        const int lanes16 = __shfl_sync(0xffffffffu, lanes16_l, r);
         const float2 mult2 = make_float2(mult, mult);
         const float2* vr = v + r * (NB / 2);
         uint8_t* row_codes = a.codes + (size_t)row * (packed4 ? K / 2 : K);
         if constexpr (kAbsmax) {
           quant_store<0, RUNS>(vr, mult2, row_codes, packed4, arow);
-        } else if (mult * sqrtf((float)NB * ssr) < 30000.f) {
+        } else if (lanes16) {
           quant_store<1, RUNS>(vr, mult2, row_codes, packed4, arow);
         } else {
           quant_store<2, RUNS>(vr, mult2, row_codes, packed4, arow);
