@@ -77,6 +77,10 @@ NFQ_CASES = [
     (8192, 0, 37, hbl.HBL_Q_A4_ABSMEAN, hbl.HBL_CODES_PACKED, False),
     (8192, 0, 7, hbl.HBL_Q_A8_ABSMAX, hbl.HBL_CODES_I8, False),
     (16384, 0, 19, hbl.HBL_Q_A4_ABSMEAN, hbl.HBL_CODES_PACKED, False),
+    # fewer rows than one group of the tensor-core kernel (16384 / K rows per group)
+    (4096, 0, 3, hbl.HBL_Q_A4_ABSMEAN, hbl.HBL_CODES_I8, False),
+    (8192, 0, 1, hbl.HBL_Q_A8_ABSMAX, hbl.HBL_CODES_PACKED, False),
+    (16384, 0, 1, hbl.HBL_Q_A4_ABSMAX, hbl.HBL_CODES_I8, False),
     (16384, 0, 3, hbl.HBL_Q_A4_ABSMEAN, hbl.HBL_CODES_I8, True),
     (768, 256, 37, hbl.HBL_Q_A4_ABSMEAN, hbl.HBL_CODES_PACKED, False),
     (11008, 256, 23, hbl.HBL_Q_A4_ABSMEAN, hbl.HBL_CODES_PACKED, False),
