@@ -38,14 +38,11 @@
 
 namespace hbl {
 
-constexpr int kNtN = 16384;                       // transform size (the whole row)
-constexpr int kNtRowBytes = kNtN * 2;             // one bf16 row
+constexpr int kNtN = 16384;                       // features in one group (16384 / K rows)
+constexpr int kNtRowBytes = kNtN * 2;             // the group's bf16 landing buffer
 constexpr int kNtThreads = 160;                   // 4 consumer warps + 1 copy / MMA warp
 constexpr int kNtTmemCols = 256;                  // two 128-column fp32 accumulators
-#ifndef HBL_NT_PAD
-#define HBL_NT_PAD 0
-#endif
-constexpr int kNtSmem = 32768 + kNtRowBytes + HBL_NT_PAD + 1024;  // H, row, alignment slack
+constexpr int kNtSmem = 32768 + kNtRowBytes + 1024;  // H, rows, alignment slack
 // CTAs resident on one SM. The copy and the MMAs of one CTA overlap the butterflies of the other,
 // so the launch sizes its grid to this many per SM. The register file is split into four
 // 16384-entry quarters, one per warp scheduler, and two 5-warp CTAs put three warps on one quarter:
