@@ -135,8 +135,9 @@ hbl_status hbl_pack_ternary(const int8_t* t, int K, int N, void* packed, size_t 
  *            be a power of two), or to each consecutive block
  *            of had_block features (block-diagonal)
  *   q, s   = quantiser `quant` applied per token row (see hbl_quant); a row whose statistic
- *            is 0 gives q = 0, s = 0. Rounding: nearest, ties to even, of the exact product of
- *            the fp32 element and the fp32 per-row multiplier (one fused multiply-add).
+ *            is 0 gives q = 0, s = 0. Rounding: nearest, ties to even. The kernels transform and
+ *            decide in fp32, so a value within fp32 rounding of a .5 boundary may land on
+ *            either side of it (a one-step code difference from an exact evaluation).
  * Kernels: one block of 4096, 8192 or 16384 features without gain runs the H_128 Kronecker factor of
  * the transform on the tensor cores and the rest on CUDA cores; every other shape runs on CUDA
  * cores. Both give the same codes up to the rounding-order ties the parity tests allow.

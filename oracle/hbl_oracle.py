@@ -20,7 +20,7 @@ pages were extracted, the surrounding words survive):
          "6 页论文，引入 1 bit LLM".
 
 Readings taken where the pages are silent or the formulas were dropped
-(each one is listed again with its reason in the design notes):
+(each is a reading of a passage whose formula was lost):
   R1 weights: per-tensor absmean alpha = mean|W|; t = RoundClip(W/(alpha+eps_w), -1, 1).
   R2 norm: RMSNorm over the K features of a token, x / sqrt(mean(x^2) + eps_n),
      optional per-feature gain; eps_n defaults to 1e-6.
@@ -32,19 +32,18 @@ Readings taken where the pages are silent or the formulas were dropped
        a4 absmean: beta = mean|x|, q = RoundClip(sqrt7 x/(beta+eps), -8, 7), s = beta/sqrt7
        a4 absmax : gamma = max|x|, q = RoundClip(7 x/(gamma+eps), -8, 7),    s = gamma/7
      A row whose statistic is zero (and eps = 0) gives q = 0 and s = 0.
-  R5 RoundClip rounds to nearest, ties to even. The rounding decision is taken
-     on float32 operands: the element and the per-row multiplier are rounded to
-     float32 and their exact product (which float64 holds without error) is
-     rounded once to an integer, as a fused multiply-add does on the GPU.
-     Everything before that is float64.
+  R5 RoundClip rounds to nearest, ties to even, and clips to the code range.
+     The pages fix no precision for any step, so every step here, the rounding
+     decision included, is taken in float64 on the float64 values of the steps
+     before it: q = clip(rint(Q * x / (stat + eps)), lo, hi).
   R6 output: y[m, n] = s[m] * alpha * sum_k q[m, k] t[k, n], evaluated in float64.
 
-Parity status: the transform, the quantisers, the ternariser and the integer
-product are pinned by the tests (closed forms, a dense Sylvester matrix from
-SciPy, brute force on small inputs, a hand-derived worked example). The
-choice of readings R1-R6 themselves is not pinned by any number on the pages,
-which print none: against the published method the oracle is "parity
-unpinned" in that sense only.
+Parity status: every function below names the tests that pin it against
+something other than itself (closed forms, a dense Sylvester matrix from
+SciPy, torch's bf16 widening, brute force on small inputs, a hand-derived
+worked example). The choice of readings R1-R6 themselves is not pinned by any
+number on the pages, which print none: against the published method the
+oracle is "parity unpinned" in that sense only.
 """
 from __future__ import annotations
 
@@ -69,9 +68,15 @@ __all__ = [
 
 
 def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
-    """bf16 bit patterns (uint16) -> float64, exactly (bf16 is the top half of a float32)."""
+    """bf16 bit patterns (uint16) -> float64, exactly (bf16 is the top half of a float32).
+
+    Pinned by test_bf16_to_f64_known_patterns (1.0, -2.0, the smallest subnormal, the largest
+    finite value, signed zero) and test_bf16_to_f64_matches_torch (all 65536 patterns against
+    torch's own bf16 -> float conversion).
+    """
     b = np.asarray(bits, dtype=np.uint16)
-    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    with np.errstate(invalid="ignore"):  # NaN patterns stay NaN
+        return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
 def absmean_ternarize(W: np.ndarray, eps_w: float = 0.0) -> tuple[np.ndarray, float]:
@@ -82,8 +87,9 @@ def absmean_ternarize(W: np.ndarray, eps_w: float = 0.0) -> tuple[np.ndarray, fl
     matrix is scaled by its mean absolute value and each entry is rounded to the
     nearest of -1, 0, 1.
 
-    Returns (t int8 with the shape of W, alpha). The rounding decision uses
-    float64 (the weight packer on the GPU also decides in float64).
+    Returns (t int8 with the shape of W, alpha); alpha does not include eps_w.
+    Pinned by test_ternarize_constant_and_brute_force (constant matrices, brute-force
+    nearest of {-1, 0, 1}, all-zero W) and test_ternarize_eps_w_closed_form.
     """
     W = np.asarray(W, dtype=np.float64)
     alpha = float(np.sum(np.abs(W)) / W.size)
@@ -100,6 +106,10 @@ def rmsnorm(x: np.ndarray, gain: np.ndarray | None = None, eps: float = 1e-6) ->
     [ART] "BitNet v2：原生4位激活": the model is built from LLaMA-like parts
     including RMS normalisation; "H-BitLinear模塊" names the normalisation
     applied inside the layer before the Hadamard transform.
+
+    Pinned by test_rmsnorm_unit_rms_and_gain (unit RMS, per-row factor, gain) and
+    test_rmsnorm_eps_under_the_square_root (a closed form that separates eps inside the
+    square root from eps added outside it or to the mean before squaring).
     """
     x = np.asarray(x, dtype=np.float64)
     r = np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
@@ -118,6 +128,9 @@ def fwht(x: np.ndarray) -> np.ndarray:
     H_2n = [[H_n, H_n], [H_n, -H_n]], realised as log2(n) butterfly stages: at
     stage h the pair (x[j], x[j+h]) inside each block of 2h becomes
     (x[j] + x[j+h], x[j] - x[j+h]). The result is scaled by 1/sqrt(n).
+
+    Pinned by test_fwht_equals_scipy_sylvester_matrix, test_fwht_walsh_closed_form,
+    test_fwht_orthogonal_involution_parseval and test_fwht_delta_and_constant.
     """
     y = np.array(x, dtype=np.float64, copy=True)
     n = y.shape[-1]
@@ -140,7 +153,9 @@ def hadamard_transform(x: np.ndarray, block: int = 0) -> np.ndarray:
 
     Block-diagonal (reading R3): K = nb * block, and each consecutive slice of
     `block` features is transformed on its own, i.e. the matrix is
-    kron(I_nb, H_block / sqrt(block)).
+    kron(I_nb, H_block / sqrt(block)). A block of 1 is the identity (H_1 = [1]).
+
+    Pinned by test_block_diagonal_transform_matches_kron and test_block_of_one_is_identity.
     """
     x = np.asarray(x, dtype=np.float64)
     K = x.shape[-1]
@@ -152,10 +167,9 @@ def hadamard_transform(x: np.ndarray, block: int = 0) -> np.ndarray:
     return fwht(x.reshape(*lead, K // block, block)).reshape(*lead, K)
 
 
-def _round_clip_f32(x: np.ndarray, mult: np.ndarray, lo: int, hi: int) -> np.ndarray:
-    """RoundClip on float32 operands (reading R5): the exact product, rounded once."""
-    v = x.astype(np.float32).astype(np.float64) * mult.astype(np.float32).astype(np.float64)  # 24 x 24 bits: exact
-    return np.clip(np.rint(v), lo, hi).astype(np.int8)  # ties to even
+def _round_clip(v: np.ndarray, lo: int, hi: int) -> np.ndarray:
+    """RoundClip (reading R5): nearest integer, ties to even, clipped to [lo, hi]."""
+    return np.clip(np.rint(v), lo, hi).astype(np.int8)
 
 
 def quantize(xr: np.ndarray, abits: int, scale_mode: str, eps_q: float = 0.0
@@ -166,7 +180,10 @@ def quantize(xr: np.ndarray, abits: int, scale_mode: str, eps_q: float = 0.0
     (formulas dropped in extraction). [B158] "6 页论文，引入 1 bit LLM":
     activations are scaled into [-Q_b, Q_b], which removes the zero point.
 
-    Returns (q int8 [M, K], s float64 [M]).
+    Returns (q int8 [M, K], s float64 [M]); s does not include eps_q.
+    Pinned by test_quantiser_defining_properties, test_quantiser_brute_force_nearest_code,
+    test_quantiser_ties_go_to_even, test_quantiser_eps_q_closed_form and
+    test_quantiser_zero_row_and_scale_invariance.
     """
     xr = np.asarray(xr, dtype=np.float64)
     a = np.abs(xr)
@@ -180,8 +197,8 @@ def quantize(xr: np.ndarray, abits: int, scale_mode: str, eps_q: float = 0.0
         raise ValueError(f"unsupported quantiser abits={abits} scale_mode={scale_mode!r}")
     denom = stat + eps_q
     live = denom > 0.0
-    mult = np.where(live, qmul / np.where(live, denom, 1.0), 0.0)
-    q = _round_clip_f32(xr, mult[..., None], lo, hi)
+    v = np.where(live[..., None], qmul * xr / np.where(live, denom, 1.0)[..., None], 0.0)
+    q = _round_clip(v, lo, hi)
     s = np.where(live, stat / qmul, 0.0)
     return q, s
 
@@ -196,6 +213,7 @@ def norm_fht_quant(x: np.ndarray, gain: np.ndarray | None, had_block: int, abits
     Q_w(W) . Q_INT8/INT4(Hadamard(LN(X))).
 
     x: float64 values (or bf16 bit patterns as uint16) [M, K].
+    Pinned through its parts and by test_worked_example (hand-derived K = 4 example).
     """
     if x.dtype == np.uint16:
         x = bf16_to_f64(x)
@@ -204,12 +222,18 @@ def norm_fht_quant(x: np.ndarray, gain: np.ndarray | None, had_block: int, abits
 
 
 def ternary_matmul(q: np.ndarray, t: np.ndarray) -> np.ndarray:
-    """acc[m, n] = sum_k q[m, k] * t[k, n] in exact int64 arithmetic (the sum written as an einsum)."""
+    """acc[m, n] = sum_k q[m, k] * t[k, n] in exact int64 arithmetic (the sum written as an einsum).
+
+    Pinned by test_ternary_matmul_brute_force_and_blas (a triple loop, float64 BLAS, np.matmul).
+    """
     return np.einsum("mk,kn->mn", np.asarray(q, dtype=np.int64), np.asarray(t, dtype=np.int64))
 
 
 def dequant(acc: np.ndarray, s: np.ndarray, alpha: float) -> np.ndarray:
-    """y[m, n] = acc[m, n] * s[m] * alpha in float64 (reading R6)."""
+    """y[m, n] = acc[m, n] * s[m] * alpha in float64 (reading R6).
+
+    Pinned by test_worked_example and test_forward_equals_dense_dequantised_product.
+    """
     return np.asarray(acc, dtype=np.float64) * np.asarray(s, dtype=np.float64)[:, None] * float(alpha)
 
 

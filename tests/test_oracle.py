@@ -81,6 +81,35 @@ def test_block_diagonal_transform_matches_kron():
         np.testing.assert_allclose(got[:, sl], x[:, sl] @ H.T, atol=1e-12)
 
 
+def test_block_of_one_is_identity():
+    # kron(I_K, H_1) with H_1 = [1]: the block-diagonal transform with blocks of one feature
+    # leaves every row unchanged (plain BitLinear, no rotation)
+    x = RNG.standard_normal((3, 768))
+    np.testing.assert_array_equal(oracle.hadamard_transform(x, 1), x)
+
+
+# ---------------------------------------------------------------- bf16 input
+
+def test_bf16_to_f64_known_patterns():
+    bits = np.array([0x3F80, 0xC000, 0x0001, 0x8001, 0x7F7F, 0x0000, 0x8000, 0x4049, 0x0080], dtype=np.uint16)
+    want = [1.0, -2.0, 2.0 ** -133, -(2.0 ** -133), (2.0 - 2.0 ** -7) * 2.0 ** 127, 0.0, -0.0,
+            3.140625, 2.0 ** -126]
+    got = oracle.bf16_to_f64(bits)
+    assert got.dtype == np.float64
+    np.testing.assert_array_equal(got, want)
+    assert math.copysign(1.0, got[6]) == -1.0
+
+
+def test_bf16_to_f64_matches_torch():
+    torch = pytest.importorskip("torch")
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    got = oracle.bf16_to_f64(bits)
+    nan = np.isnan(ref)
+    np.testing.assert_array_equal(np.isnan(got), nan)
+    np.testing.assert_array_equal(got[~nan], ref[~nan])
+
+
 # ---------------------------------------------------------------- norm
 
 def test_rmsnorm_unit_rms_and_gain():
@@ -94,6 +123,18 @@ def test_rmsnorm_unit_rms_and_gain():
     np.testing.assert_allclose(oracle.rmsnorm(x, g, eps=0.0), y * g, rtol=1e-13)
     # eps enters under the square root: a zero row stays zero
     np.testing.assert_array_equal(oracle.rmsnorm(np.zeros((1, 8)), None, 1e-6), np.zeros((1, 8)))
+
+
+def test_rmsnorm_eps_under_the_square_root():
+    # x = [3, 4]: mean(x^2) = 12.5. With eps = 11.5 under the square root r = sqrt(24), so
+    # y = [3, 4] / sqrt(24). Eps added outside the root would give r = sqrt(12.5) + 11.5, eps on
+    # the mean before squaring something else again; both differ here by far more than rounding.
+    y = oracle.rmsnorm(np.array([[3.0, 4.0]]), None, eps=11.5)
+    np.testing.assert_allclose(y[0], np.array([3.0, 4.0]) / math.sqrt(24.0), rtol=1e-15)
+    assert abs(y[0, 0] - 3.0 / (math.sqrt(12.5) + 11.5)) > 0.1
+    # the gain multiplies after the division
+    y = oracle.rmsnorm(np.array([[3.0, 4.0]]), np.array([2.0, -1.0]), eps=11.5)
+    np.testing.assert_allclose(y[0], np.array([6.0, -4.0]) / math.sqrt(24.0), rtol=1e-15)
 
 
 def test_rms_is_preserved_by_the_orthonormal_transform():
@@ -128,28 +169,53 @@ def test_quantiser_defining_properties(abits, mode, Q, lo, hi):
         np.testing.assert_array_equal(np.abs(q[np.arange(64), am]), int(Q))
 
 
-def test_rounding_takes_the_exact_product():
-    # x = 1 + 2^-23 and mult = 2.5 - 2^-22 are float32 values whose exact product is
-    # 2.5 + 2^-24 - 2^-45: just above the tie, so the code is 3. Rounding the product to float32
-    # first would land exactly on 2.5 and give the even code 2.
-    x = np.array([1.0 + 2.0 ** -23])
-    mult = np.array([2.5 - 2.0 ** -22])
-    assert np.float32(x[0]) == x[0] and np.float32(mult[0]) == mult[0]
-    assert float(np.float32(x[0]) * np.float32(mult[0])) == 2.5
-    assert oracle.hbl_oracle._round_clip_f32(x, mult, -8, 7)[0] == 3
+def test_quantiser_ties_go_to_even():
+    # exact ties in float64: a4 absmax with gamma = 7 maps x to x itself, so x = +-2.5, 3.5, 0.5
+    # sit on .5 boundaries; nearest-even gives 2, 4, 0 (round-half-away would give 3, 4, 1,
+    # floor 2, 3, 0, and a float32 detour cannot move them: every value here is exact)
+    x = np.array([[2.5, -2.5, 3.5, 0.5, -0.5, 7.0]])
+    q, s = oracle.quantize(x, 4, "absmax")
+    np.testing.assert_array_equal(q[0], [2, -2, 4, 0, 0, 7])
+    assert s[0] == 1.0
+    # a8 absmax: gamma = 127 maps x to x; 126.5 -> 126, -127.5 cannot occur (|x| <= gamma)
+    x = np.array([[126.5, -1.5, 127.0, 64.5]])
+    q, _ = oracle.quantize(x, 8, "absmax")
+    np.testing.assert_array_equal(q[0], [126, -2, 127, 64])
+
+
+def test_quantiser_eps_q_closed_form():
+    # reading R4 with eps: q = RoundClip(Q x / (stat + eps), lo, hi), s = stat / Q (no eps in s)
+    x = np.array([[1.0, -2.0, 3.0, -4.0]])
+    # a4 absmean: beta = 2.5; eps = 1.5 gives multiplier sqrt7 / 4 = 0.6614...:
+    # [0.661, -1.323, 1.984, -2.646] -> [1, -1, 2, -3]; without eps sqrt7 / 2.5 gives [1, -2, 3, -4]
+    q, s = oracle.quantize(x, 4, "absmean", eps_q=1.5)
+    np.testing.assert_array_equal(q[0], [1, -1, 2, -3])
+    assert s[0] == pytest.approx(2.5 / math.sqrt(7), rel=1e-15)
+    q0, _ = oracle.quantize(x, 4, "absmean")
+    np.testing.assert_array_equal(q0[0], [1, -2, 3, -4])
+    # a8 absmax: gamma = 4, eps = 1: 127 x / 5 = [25.4, -50.8, 76.2, -101.6] -> [25, -51, 76, -102]
+    q, s = oracle.quantize(x, 8, "absmax", eps_q=1.0)
+    np.testing.assert_array_equal(q[0], [25, -51, 76, -102])
+    assert s[0] == pytest.approx(4.0 / 127.0, rel=1e-15)
+    # a4 absmax: gamma = 4, eps = 4: 7 x / 8 = [0.875, -1.75, 2.625, -3.5] -> [1, -2, 3, -4] (-3.5 is a tie: even)
+    q, _ = oracle.quantize(x, 4, "absmax", eps_q=4.0)
+    np.testing.assert_array_equal(q[0], [1, -2, 3, -4])
+    # with eps > 0 a zero row is still all zeros, with s = 0
+    q, s = oracle.quantize(np.zeros((1, 4)), 4, "absmean", eps_q=0.5)
+    assert not q.any() and s[0] == 0.0
 
 
 @pytest.mark.parametrize("abits,mode,Q,lo,hi", QUANTS)
 def test_quantiser_brute_force_nearest_code(abits, mode, Q, lo, hi):
-    # brute force: among all codes in [lo, hi] the oracle picks the one nearest to the exact
-    # product of the float32 element and the float32 multiplier (ties to the even code).
+    # brute force: among all codes in [lo, hi] the oracle picks the one nearest to Q x / stat
+    # (ties to the even code), found here by searching every code rather than rounding.
     x = RNG.standard_normal((8, 32))
     q, s = oracle.quantize(x, abits, mode)
-    stat = np.abs(x).max(axis=1) if mode == "absmax" else np.abs(x).mean(axis=1)
     for m in range(8):
-        mult = np.float32(Q / stat[m])
+        row = [abs(float(v)) for v in x[m]]
+        stat = max(row) if mode == "absmax" else sum(row) / len(row)
         for k in range(32):
-            vv = float(np.float32(x[m, k])) * float(mult)  # exact in a Python float
+            vv = Q * float(x[m, k]) / stat
             best = min(range(lo, hi + 1), key=lambda c: (abs(vv - c), c % 2))
             assert q[m, k] == best, (m, k, vv, q[m, k], best)
 
@@ -188,6 +254,22 @@ def test_ternarize_constant_and_brute_force():
         assert t[k, n] == best
     t0, a0 = oracle.absmean_ternarize(np.zeros((3, 3)))
     assert a0 == 0.0 and not t0.any()
+
+
+def test_ternarize_eps_w_closed_form():
+    # alpha = mean|W| = 1.0 / 4 = 0.25. Without eps W / alpha = [0.8, -1.2, 2.0, 0] -> [1, -1, 1, 0];
+    # with eps_w = 0.2 the divisor is 0.45: [0.444, -0.667, 1.11, 0] -> [0, -1, 1, 0]. alpha itself
+    # does not include eps.
+    W = np.array([[0.2, -0.3], [0.5, 0.0]])
+    t, alpha = oracle.absmean_ternarize(W)
+    np.testing.assert_array_equal(t, [[1, -1], [1, 0]])
+    assert alpha == pytest.approx(0.25, rel=1e-15)
+    t, alpha = oracle.absmean_ternarize(W, eps_w=0.2)
+    np.testing.assert_array_equal(t, [[0, -1], [1, 0]])
+    assert alpha == pytest.approx(0.25, rel=1e-15)
+    # an all-zero W with eps > 0 gives t = 0 as well
+    t, alpha = oracle.absmean_ternarize(np.zeros((2, 2)), eps_w=0.1)
+    assert not t.any() and alpha == 0.0
 
 
 # ---------------------------------------------------------------- product
@@ -298,3 +380,24 @@ def test_planted_quantiser_mistake_is_caught(monkeypatch):
     monkeypatch.setattr(oracle, "quantize", floor_instead_of_round)
     with pytest.raises(AssertionError):
         test_quantiser_defining_properties(4, "absmean", math.sqrt(7), -8, 7)
+
+
+def test_planted_norm_and_rounding_mistakes_are_caught(monkeypatch):
+    real_rms = oracle.hbl_oracle.rmsnorm
+
+    def eps_outside_root(x, gain=None, eps=1e-6):
+        x = np.asarray(x, dtype=np.float64)
+        y = x / (np.sqrt(np.mean(x * x, axis=-1, keepdims=True)) + eps)
+        return y if gain is None else y * gain
+
+    monkeypatch.setattr(oracle, "rmsnorm", eps_outside_root)
+    with pytest.raises(AssertionError):
+        test_rmsnorm_eps_under_the_square_root()
+    monkeypatch.setattr(oracle, "rmsnorm", real_rms)
+
+    def half_away(v, lo, hi):
+        return np.clip(np.sign(v) * np.floor(np.abs(v) + 0.5), lo, hi).astype(np.int8)
+
+    monkeypatch.setattr(oracle.hbl_oracle, "_round_clip", half_away)
+    with pytest.raises(AssertionError):
+        test_quantiser_ties_go_to_even()
