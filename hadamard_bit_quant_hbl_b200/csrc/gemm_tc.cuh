@@ -107,6 +107,4 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
       : "memory");
 }
 
-// ---------------------------------------------------------------- the kernel
-
 }  // namespace hbl

@@ -687,8 +687,11 @@ StaticScratch& static_scratch() {
   return s;
 }
 
-// Device address of g_static_scratch on the current device (looked up once per device; host
-// code only sees a host-side stand-in for the array's name, never its device address).
+// Device address of g_static_scratch on the current device. Host code only sees a host-side
+// stand-in for the array's name, never its device address, so the address is looked up with
+// cudaGetSymbolAddress once per device (on the first call there) and kept for the life of the
+// process. It belongs to the device's primary context: after that context is destroyed
+// (cudaDeviceReset) the kept address is stale, which hbl.h states as a limit of this entry point.
 hbl_status static_scratch_addr(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -714,7 +717,7 @@ extern "C" hbl_status hbl_forward_static(const void* X, const float* gain, const
                                          void* Y, hbl_out_dtype out_dtype, hbl_stream_t stream) {
   if (!dims_ok(M, K)) return HBL_EINVAL;
   const size_t need = hbl_forward_workspace(M, K, quant);
-  if (need > kStaticScratchBytes) return HBL_EINVAL;  // request larger than the static scratch
+  if (need > kStaticScratchBytes) return HBL_EUNSUPPORTED;  // request larger than the static scratch
   void* ws = nullptr;
   const hbl_status st = static_scratch_addr(&ws);
   if (st != HBL_OK) return st;

@@ -198,9 +198,12 @@ hbl_status hbl_forward(const void* X, const float* gain, const void* packed, siz
  * inside the library's device image (a static __device__ array): every GPU that loads the library
  * holds those 16 MiB until the process exits, and no call allocates or frees device memory.
  *   - Requests needing more than 16 MiB of scratch (roughly M * K > 16.7 million) return
- *     HBL_EINVAL; use hbl_forward with your own workspace for them.
+ *     HBL_EUNSUPPORTED before any device work; use hbl_forward with your own workspace for them.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
- *     with that device current; make that first call before any stream capture.
+ *     with that device current and keeps it for the life of the process; make that first call
+ *     before any stream capture. Resetting the device (cudaDeviceReset, or any other teardown of
+ *     its primary context) after that first call is not supported: the kept address would be
+ *     stale.
  *   - All calls on a device share the one array, and each call leaves its scratch contents
  *     behind. Calls that may overlap on the GPU (different streams without ordering between
  *     them) race on it: serialise them, or use hbl_forward.

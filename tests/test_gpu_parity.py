@@ -89,6 +89,14 @@ NFQ_CASES = [
     (12288, 4096, 6, hbl.HBL_Q_A4_ABSMEAN, hbl.HBL_CODES_PACKED, False),
     (32768, 16384, 3, hbl.HBL_Q_A4_ABSMEAN, hbl.HBL_CODES_PACKED, False),
     (32768, 256, 3, hbl.HBL_Q_A4_ABSMEAN, hbl.HBL_CODES_PACKED, False),
+    # more row groups than resident CTAs (two per SM): every CTA of the tensor-core kernel walks
+    # three or more groups, through both TMEM accumulators and the refill of its copy buffer
+    (16384, 0, 1000, hbl.HBL_Q_A4_ABSMEAN, hbl.HBL_CODES_I8, False),
+    (8192, 0, 2000, hbl.HBL_Q_A4_ABSMAX, hbl.HBL_CODES_PACKED, False),
+    (4096, 0, 4000, hbl.HBL_Q_A8_ABSMAX, hbl.HBL_CODES_I8, False),
+    # and the CUDA-core kernel over thousands of row groups
+    (2048, 0, 3000, hbl.HBL_Q_A4_ABSMEAN, hbl.HBL_CODES_I8, False),
+    (11008, 256, 700, hbl.HBL_Q_A4_ABSMEAN, hbl.HBL_CODES_I8, False),
 ]
 
 
@@ -210,6 +218,10 @@ GEMM_CASES = [
     (300, 2048, 520, 4, hbl.HBL_CODES_I8),
     (257, 11008, 264, 4, hbl.HBL_CODES_I8),
     (200, 4096, 1032, 8, hbl.HBL_CODES_I8),
+    # more 256 x 256 pair tiles than SM pairs: clusters walk two or more tiles, alternating their
+    # two TMEM accumulators (80 and 160 tiles for 74 pairs)
+    (2560, 512, 2048, 4, hbl.HBL_CODES_I8),
+    (2560, 256, 4096, 8, hbl.HBL_CODES_I8),
 ]
 
 
@@ -311,6 +323,23 @@ def test_forward_full_size_sampled_rows(name, M):
     picks = [0, 1, spec.M // 2, spec.M - 1] + list(np.random.default_rng(spec.M).integers(0, spec.M, 4))
     rows = sorted(set(int(r) for r in picks if r < spec.M))
     check_forward(spec, rows=rows, out_dtype=hbl.HBL_OUT_BF16)
+
+
+@pytest.mark.parametrize("name,M", [("wdown_7b_a4", 8192), ("wo_7b_a4", 8192)])
+def test_norm_fht_quant_full_size_every_row(name, M):
+    # the activation kernel exactly as the benchmark launches it (a4 absmean, int8 codes) at full
+    # size: every code and every scale against the oracle, rows checked in chunks
+    spec = inputs.WORKLOADS[name].with_m(M)
+    x = inputs.activations(spec)
+    q, s = gpu_codes(x, None, spec.had_block, hbl.HBL_Q_A4_ABSMEAN, hbl.HBL_CODES_I8)
+    flips = 0
+    for r0 in range(0, M, 1024):
+        q_ref, s_ref = oracle.norm_fht_quant(x[r0:r0 + 1024], None, spec.had_block, 4, "absmean")
+        d = np.abs(q[r0:r0 + 1024].astype(np.int32) - q_ref)
+        assert d.max() <= 1
+        flips += int(np.count_nonzero(d))
+        np.testing.assert_allclose(s[r0:r0 + 1024], s_ref, rtol=1e-5)
+    assert flips <= max(1, int(1e-4 * M * spec.K)), flips
 
 
 @pytest.mark.parametrize("M", [1, 3, 16, 64, 300])

@@ -29,11 +29,13 @@ def _entry():
 
 
 def test_static_forward_rejects_requests_beyond_its_scratch():
-    # 1024 x 32768 needs 32 MiB of scratch: refused before any device work
+    # 1024 x 32768 needs 32 MiB of scratch: refused with its own status before any device work.
+    # Every pointer is NULL, so if the size check ever stopped refusing, the call would return
+    # HBL_EINVAL from the pointer checks instead (and still launch nothing).
     f = _entry()
-    st = f(1 << 20, None, 1 << 20, 1 << 30, 1.0, 1024, 32768, 64, 0, hbl.HBL_Q_A4_ABSMEAN, 1e-6, 0.0, 1 << 20,
+    st = f(None, None, None, 0, 1.0, 1024, 32768, 64, 0, hbl.HBL_Q_A4_ABSMEAN, 1e-6, 0.0, None,
            hbl.HBL_OUT_F32, None)
-    assert st == hbl.HBL_EINVAL
+    assert st == hbl.HBL_EUNSUPPORTED, hbl.hbl_status_string(st)
 
 
 @pytest.mark.gpu
@@ -45,8 +47,9 @@ def test_static_forward_matches_forward_on_two_calls():
     torch.cuda.set_device(0)
     f = _entry()
     stream = torch.cuda.current_stream().cuda_stream
-    cases = [("wdown_3b_a4", 300, hbl.HBL_OUT_F32),   # tensor-core product
-             ("wo_7b_a4", 5, hbl.HBL_OUT_BF16)]       # CUDA-core product
+    cases = [("wdown_3b_a4", 300, hbl.HBL_OUT_F32),   # SM-pair tensor-core product
+             ("wo_7b_a4", 5, hbl.HBL_OUT_BF16),       # swapped-operand tensor-core product
+             ("wdown_7b_a4", 3, hbl.HBL_OUT_F32)]     # CUDA-core product (int8 codes, M <= 4)
     results = []
     for name, M, out_dtype in cases:
         spec = inputs.WORKLOADS[name].with_m(M)
