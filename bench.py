@@ -37,10 +37,10 @@ LAYERS = ("wo_7b_a4", "wdown_7b_a4")
 SWEEP_TOKENS = (1, 16, 64, 512)
 WORKLOAD = ("7B-like H-BitLinear layer pair: Wo 4096->4096 + Wdown 16384->4096, a4 absmean, "
             "8192 tokens, bf16 in / bf16 out")
-# DRAM bytes per launch of the dominant kernel from an ncu capture, with the hash of the kernel
-# source it was taken on (reported as null once the source has changed).
+# DRAM bytes per launch of the dominant kernel (dram__bytes_read.sum + dram__bytes_write.sum from
+# one ncu capture of the Wdown product at 8192 tokens), with the hash of the kernel source it was
+# taken on (reported as null once the source has changed).
 NCU_TRAFFIC = {
-    # profiles/gemm_tc2_wdown_7b_m8192.md: dram__bytes_read.sum + dram__bytes_write.sum
     "gemm_tc2[wdown_7b_a4]": {"bytes": 600.112896e6 + 69.806592e6, "src": "gemm_tc2.cuh", "sha": "2cc3da467c32c2e2"},
 }
 
@@ -54,7 +54,21 @@ def product_kernel(M):
 
 def nfq_kernel(K, had_block):
     """Name of the fused activation kernel hbl_norm_fht_quant runs (no gain)."""
+    if had_block == 1:
+        return "norm_quant"
     return "norm_fht_quant_tc" if (K in (4096, 8192, 16384) and had_block == 0) else "norm_fht_quant"
+
+
+def act_bytes(M, K, abits):
+    """Algorithmic HBM bytes of the fused activation step: the bf16 input, the codes at their
+    bit width (a4: half a byte per feature), one fp32 scale per row."""
+    return 2 * M * K + (M * K * abits) // 8 + 4 * M
+
+
+def act_container_bytes(M, K):
+    """Bytes the activation kernel moves when it writes one int8 container per code (the format
+    the tensor-core products read)."""
+    return 2 * M * K + M * K + 4 * M
 
 
 def weight_bytes(M, K, N):
@@ -172,6 +186,98 @@ def oracle_step(prepared):
         q, s = oracle.norm_fht_quant(x, None, spec.had_block, 4, "absmean")
         oracle.dequant(oracle.ternary_matmul(q, t), s, alpha)
     return time.perf_counter() - t0
+
+
+# The oracle on all host cores: a spawned process pool (never forked from a process that has
+# used the GPU), each worker mapping the ternarised weights and the sample rows from files, and
+# running S1-S3 then S4-S5 on a slice of rows.
+_CPU_DATA = {}
+
+
+def _cpu_init(files):
+    global _CPU_DATA
+    import oracle  # noqa: F401  (imported before timing)
+
+    _CPU_DATA = {name: (np.load(tp, mmap_mode="r"), alpha, np.load(xp, mmap_mode="r"), had)
+                 for name, (tp, alpha, xp, had) in files.items()}
+
+
+def _cpu_task(task):
+    import oracle
+
+    name, r0, r1 = task
+    t, alpha, x, had = _CPU_DATA[name]
+    t0 = time.perf_counter()
+    q, s = oracle.norm_fht_quant(np.array(x[r0:r1]), None, had, 4, "absmean")
+    t1 = time.perf_counter()
+    oracle.dequant(oracle.ternary_matmul(q, t), s, alpha)
+    return t1 - t0, time.perf_counter() - t1
+
+
+def cpu_baseline(rows_one_core):
+    """Times the oracle, as it stands, on the host: on one core over the first `rows_one_core`
+    token rows of each layer, and on all available cores (one worker process per core, capped by
+    free memory: each worker widens the ternary weights to int64) over `rows_one_core` rows per
+    worker and layer. S1-S3 (norm, transform, quantise) and S4-S5 (integer product, dequant) are
+    timed separately. Returns the cpu_baseline object of the bench line (its value: all cores)."""
+    import multiprocessing as mp
+    import shutil
+    import tempfile
+
+    import oracle
+
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    try:
+        import psutil
+
+        cores = max(1, min(cores, int(psutil.virtual_memory().available / 1.5e9)))
+    except Exception:
+        pass
+    rows_all = rows_one_core * cores
+    tmp = tempfile.mkdtemp(prefix="hbl_oracle_")
+    try:
+        files, prepared = {}, []
+        for name in LAYERS:
+            spec = inputs.WORKLOADS[name].with_m(rows_all)
+            t, alpha = oracle.absmean_ternarize(inputs.weights(spec))
+            x = inputs.activations(spec)
+            tp, xp = os.path.join(tmp, f"{name}_t.npy"), os.path.join(tmp, f"{name}_x.npy")
+            np.save(tp, t)
+            np.save(xp, x)
+            files[name] = (tp, alpha, xp, spec.had_block)
+            prepared.append((name, t, alpha, x[:rows_one_core], spec.had_block))
+        # one core, in this process
+        t13 = t45 = 0.0
+        for name, t, alpha, x, had in prepared:
+            t0 = time.perf_counter()
+            q, s_ = oracle.norm_fht_quant(x, None, had, 4, "absmean")
+            t1 = time.perf_counter()
+            oracle.dequant(oracle.ternary_matmul(q, t), s_, alpha)
+            t13 += t1 - t0
+            t45 += time.perf_counter() - t1
+        del prepared
+        one = {"value": rows_one_core / (t13 + t45), "unit": UNIT, "cores": 1,
+               "s1_s3_s": t13, "s4_s5_s": t45,
+               "sample": f"first {rows_one_core} token rows of each layer"}
+        # all cores: slices of rows_one_core rows, one per worker and layer
+        tasks = [(name, r0, r0 + rows_one_core) for name in LAYERS for r0 in range(0, rows_all, rows_one_core)]
+        with mp.get_context("spawn").Pool(cores, initializer=_cpu_init, initargs=(files,)) as pool:
+            pool.map(_cpu_task, [(LAYERS[0], 0, 1)] * cores)  # workers up (imports, file maps)
+            w0 = time.perf_counter()
+            parts = pool.map(_cpu_task, tasks, chunksize=1)
+            wall = time.perf_counter() - w0
+        busy13 = sum(p[0] for p in parts)
+        busy45 = sum(p[1] for p in parts)
+        return {"value": rows_all / wall, "unit": UNIT, "cores": cores, "kind": "oracle",
+                "sample": f"first {rows_all} token rows of each layer ({rows_one_core} per worker and layer), "
+                          f"S1-S5 with weights ternarised before timing, {wall:.1f} s on {cores} worker processes",
+                "s1_s3_share": busy13 / (busy13 + busy45), "s4_s5_share": busy45 / (busy13 + busy45),
+                "one_core": one}
+    finally:
+        shutil.rmtree(tmp, ignore_errors=True)
 
 
 def run_reference(args, world, rank):
@@ -336,6 +442,9 @@ def run_ours(args, world, rank, local):
 
     # ---- token-count sweep of the same layer pair (CUDA-graph replay over rotating weight copies)
     sweep = [] if args.no_sweep else run_sweep(layers, dev, args)
+    hbm, bf16, bf16_sus, peak_src = peaks()
+    int8_peak_tops = 2.0 * bf16  # burst bf16 x nominal dense int8:bf16 ratio (4.5 : 2.25 PFLOP/s)
+    configs = [] if args.no_configs else time_configs(dev, hbm, int8_peak_tops)
 
     st = hbl.hbl_device_status()
     if st != hbl.HBL_OK:
@@ -343,16 +452,17 @@ def run_ours(args, world, rank, local):
     if rank != 0:
         return
 
-    hbm, bf16, bf16_sus, peak_src = peaks()
-    int8_peak_tops = 2.0 * bf16  # burst bf16 x nominal dense int8:bf16 ratio (4.5 : 2.25 PFLOP/s)
     kern = []
     for i, L in enumerate(layers):
         sp = L["spec"]
-        nfq_bytes = 2 * sp.M * sp.K + sp.M * sp.K + 4 * sp.M
+        nfq_bytes = act_bytes(sp.M, sp.K, 4)
         gemm_ops = 2.0 * sp.M * sp.N * sp.K
         kern.append({"kernel": f"{nfq_kernel(sp.K, sp.had_block)}[{sp.name}]", "ms": per[2 * i], "bound": "hbm",
                      "achieved": nfq_bytes / (per[2 * i] / 1e3) / 1e9, "unit": "GB/s",
-                     "frac": nfq_bytes / (per[2 * i] / 1e3) / 1e9 / hbm})
+                     "frac": nfq_bytes / (per[2 * i] / 1e3) / 1e9 / hbm, "algorithmic_bytes": nfq_bytes,
+                     "moved_bytes": act_container_bytes(sp.M, sp.K),
+                     "note": "frac on a4 algorithmic bytes (packed int4 codes); the kernel writes one int8 "
+                             "container per code, moved_bytes - algorithmic_bytes is that overhead"})
         kern.append({"kernel": f"{product_kernel(sp.M)[0]}[{sp.name}]", "ms": per[2 * i + 1], "bound": "tensor",
                      "achieved": gemm_ops / (per[2 * i + 1] / 1e3) / 1e12, "unit": "TOP/s",
                      "frac": gemm_ops / (per[2 * i + 1] / 1e3) / 1e12 / int8_peak_tops})
@@ -366,11 +476,7 @@ def run_ours(args, world, rank, local):
     # CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        rows = args.ref_rows
-        dt = oracle_step(oracle_prepare(rows))
-        cpu = {"value": rows / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"first {rows} token rows of each layer, S1-S5 (weights ternarised before timing), "
-                         f"{dt:.1f} s on one host core"}
+        cpu = cpu_baseline(args.ref_rows)
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -392,6 +498,7 @@ def run_ours(args, world, rank, local):
                  "d2h_bytes_per_step": d2h} if e2e_steps else None),
         "gpu_launches": 4 * args.steps,
         "sweep": sweep,
+        "configs": configs,
         "clocks": clk.summary(),
         "cpu_baseline": cpu,
     }
@@ -456,6 +563,78 @@ def run_sweep(layers, dev, args):
     return out
 
 
+CONFIG_CASES = [("wo_1p3b_a4", "1.3B-like Wo a4, 2048 x 2048 -> 2048"),
+                ("wdown_3b_a4", "3B-like Wdown a4, 4096 x 8192 -> 2560"),
+                ("wdown_nonpow2_a4", "Wdown a4 with block-diagonal transform (43 x 256), 8192 x 11008 -> 4096")]
+
+
+def time_configs(dev, hbm, int8_peak, reps=20):
+    """CUDA-event times of the activation kernel and of the product kernel, each launched alone
+    on its own stream, for the other full-size workloads. Every launch works on the next of
+    several copies of its inputs and outputs whose total exceeds L2."""
+    import torch
+
+    import hadamard_bit_quant_hbl_b200 as hbl
+
+    out = []
+    s = torch.cuda.Stream(dev)
+    for name, label in CONFIG_CASES:
+        spec = inputs.WORKLOADS[name]
+        M, K, N = spec.M, spec.K, spec.N
+        quant = hbl.HBL_Q_A8_ABSMAX if spec.abits == 8 else hbl.HBL_Q_A4_ABSMEAN
+        X0 = torch.from_numpy(inputs.activations(spec).view(np.int16)).to(dev).view(torch.bfloat16)
+        p0, alpha = hbl.hbl_pack_weights(torch.from_numpy(inputs.weights(spec)).to(dev))
+        nb_act = 3 * M * K + 4 * M
+        nb_prod = M * K + p0.numel() + 2 * M * N
+        na = max(2, -(-400_000_000 // nb_act))
+        npd = max(2, -(-400_000_000 // nb_prod))
+        acts = [(X0 if i == 0 else X0.clone(), torch.empty((M, K), dtype=torch.uint8, device=dev),
+                 torch.empty(M, dtype=torch.float32, device=dev)) for i in range(na)]
+        prods = [(acts[i % na][1], acts[i % na][2], p0 if i == 0 else p0.clone(),
+                  torch.empty((M, N), dtype=torch.bfloat16, device=dev)) for i in range(npd)]
+
+        def act(j):
+            X, codes, sx = acts[j % na]
+            hbl.hbl_norm_fht_quant(X, None, spec.had_block, quant, 1e-6, 0.0, hbl.HBL_CODES_I8, codes, sx,
+                                   stream=s.cuda_stream)
+
+        def prod(j):
+            codes, sx, packed, Y = prods[j % npd]
+            hbl.hbl_ternary_gemm(codes, hbl.HBL_CODES_I8, spec.abits, sx, packed, alpha, N, K, Y, hbl.HBL_OUT_BF16,
+                                 None, stream=s.cuda_stream)
+
+        res = {}
+        with torch.cuda.stream(s):
+            for j in range(na):
+                act(j)  # every codes buffer written before the products read them
+            for fn, key in ((act, "act"), (prod, "prod")):
+                for j in range(3):
+                    fn(j)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(s)
+                for j in range(reps):
+                    fn(j)
+                e1.record(s)
+                e1.synchronize()
+                res[key] = e0.elapsed_time(e1) / reps * 1e3  # us
+        st = hbl.hbl_device_status()
+        if st != hbl.HBL_OK:
+            raise RuntimeError(hbl.hbl_status_string(st))
+        ab = act_bytes(M, K, spec.abits)
+        ops = 2.0 * M * N * K
+        out.append({
+            "config": label, "M": M, "K": K, "N": N, "had_block": spec.had_block,
+            "activation": {"kernel": nfq_kernel(K, spec.had_block), "us": res["act"], "bound": "hbm",
+                           "algorithmic_bytes": ab, "moved_bytes": act_container_bytes(M, K),
+                           "GBps": ab / res["act"] / 1e3, "frac": ab / res["act"] / 1e3 / hbm},
+            "product": {"kernel": product_kernel(M)[0], "us": res["prod"], "bound": "tensor",
+                        "TOPs": ops / res["prod"] / 1e6, "frac": ops / res["prod"] / 1e6 / int8_peak},
+            "forward_us": res["act"] + res["prod"], "tokens_per_s": M / ((res["act"] + res["prod"]) / 1e6),
+            "l2": f"{na} activation and {npd} product input copies rotated"})
+        del acts, prods, X0, p0
+    return out
+
+
 def run_profile_product(M):
     """Runs the activation kernel once and the product three times on the Wdown shape with M
     tokens (a small, self-contained target for an ncu capture of one product kernel)."""
@@ -478,15 +657,15 @@ def run_profile_product(M):
 
 
 ACTIVATION_CASES = [("wo_7b_a4", 8192), ("wdown_7b_a4", 8192), ("wdown_3b_a4", 4096),
-                    ("wdown_nonpow2_a4", 8192), ("wo_1p3b_a4", 2048)]
+                    ("wdown_nonpow2_a4", 8192), ("wo_1p3b_a4", 2048), ("qkv_7b_plain_a4", 8192)]
 
 
 def run_activation_only(reps=50):
     """Times the fused activation kernel (hbl_norm_fht_quant, a4 absmean, int8 codes) alone on
     each workload width, with CUDA events on its stream. Each launch works on the next of several
     input/output copies whose total exceeds L2, so that no launch finds its data in L2. Prints one
-    line per workload (algorithmic bytes: the bf16 input, one code byte per feature, one scale per
-    row); no bench line."""
+    line per workload with the rate on the algorithmic bytes (the bf16 input, half a byte per a4
+    code, one scale per row) and on the bytes moved (one int8 container per code); no bench line."""
     import torch
 
     import hadamard_bit_quant_hbl_b200 as hbl
@@ -523,9 +702,11 @@ def run_activation_only(reps=50):
             raise RuntimeError(hbl.hbl_status_string(st))
         us = e0.elapsed_time(e1) / reps * 1000
         kern = nfq_kernel(K, spec.had_block)
+        ab = act_bytes(M, K, spec.abits)
         print(f"{kern:18s} {name:18s} M={M:5d} K={K:6d} had_block={spec.had_block:4d} {us:8.1f} us "
-              f"{nbytes / us / 1e3:7.1f} GB/s {nbytes / us / 1e3 / peak:6.3f} of {peak_src} HBM "
-              f"({ncopy} copies rotated)", flush=True)
+              f"{ab / us / 1e3:7.1f} GB/s {ab / us / 1e3 / peak:6.3f} of {peak_src} HBM on a4 algorithmic bytes "
+              f"({nbytes / us / 1e3 / peak:6.3f} on the int8-container bytes moved; {ncopy} copies rotated)",
+              flush=True)
         del bufs
 
 
@@ -535,12 +716,14 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--ref-rows", type=int, default=64, help="token rows per layer in the CPU-baseline sample")
+    ap.add_argument("--ref-rows", type=int, default=32,
+                    help="token rows per layer in the one-core CPU-baseline sample (and per worker on all cores)")
     ap.add_argument("--ref-step-rows", type=int, default=1, help="token rows per layer in one reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--no-sweep", action="store_true", help="skip the token-count sweep")
     ap.add_argument("--sweep-steps", type=int, default=100)
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-kernel times of the other workloads")
     ap.add_argument("--profile-product", type=int, default=0, metavar="M",
                     help="only run the Wdown product three times with M tokens (an ncu target); no bench line")
     ap.add_argument("--activation-only", action="store_true",

@@ -21,8 +21,10 @@ __all__ = [
     "HBL_CODES_PACKED", "HBL_CODES_I8", "HBL_OUT_F32", "HBL_OUT_BF16",
     "HblError", "lib", "library_path",
     "hbl_status_string", "hbl_device_status", "hbl_selftest_timeout", "hbl_packed_weights_bytes", "hbl_pack_weights_workspace",
-    "hbl_pack_weights", "hbl_pack_ternary", "hbl_norm_fht_quant", "hbl_ternary_gemm",
+    "hbl_pack_weights", "hbl_pack_weights_rotated", "hbl_pack_weights_rotated_workspace", "hbl_pack_ternary",
+    "hbl_norm_fht_quant", "hbl_ternary_gemm",
     "hbl_forward_workspace", "hbl_forward", "codes_row_bytes",
+    "hbl_qkv_codes_bytes", "hbl_qkv_quant", "hbl_qkv_dequant",
 ]
 
 HBL_OK, HBL_EINVAL, HBL_EUNSUPPORTED, HBL_ECUDA, HBL_ETIMEOUT = range(5)
@@ -50,12 +52,19 @@ _SIGNATURES = {
     "hbl_pack_weights_workspace": (_c_size_t, [_c_int, _c_int]),
     "hbl_pack_weights": (_c_int, [_c_void_p, _c_int, _c_int, _c_float, _c_void_p, _c_size_t,
                                   ctypes.POINTER(_c_float), _c_void_p, _c_size_t, _c_void_p]),
+    "hbl_pack_weights_rotated_workspace": (_c_size_t, [_c_int, _c_int]),
+    "hbl_pack_weights_rotated": (_c_int, [_c_void_p, _c_int, _c_int, _c_int, _c_float, _c_void_p, _c_size_t,
+                                          ctypes.POINTER(_c_float), _c_void_p, _c_size_t, _c_void_p]),
     "hbl_pack_ternary": (_c_int, [_c_void_p, _c_int, _c_int, _c_void_p, _c_size_t, _c_void_p]),
     "hbl_norm_fht_quant": (_c_int, [_c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_float,
                                     _c_float, _c_int, _c_void_p, _c_void_p, _c_void_p]),
     "hbl_ternary_gemm": (_c_int, [_c_void_p, _c_int, _c_int, _c_void_p, _c_void_p, _c_size_t, _c_float,
                                   _c_int, _c_int, _c_int, _c_void_p, _c_int, _c_void_p, _c_void_p]),
     "hbl_forward_workspace": (_c_size_t, [_c_int, _c_int, _c_int]),
+    "hbl_qkv_codes_bytes": (_c_size_t, [_c_int, _c_int, _c_int, _c_int]),
+    "hbl_qkv_quant": (_c_int, [_c_void_p, _c_size_t, _c_void_p, _c_float, _c_int, _c_int, _c_int, _c_int, _c_void_p,
+                               _c_size_t, _c_void_p, _c_void_p]),
+    "hbl_qkv_dequant": (_c_int, [_c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_void_p, _c_void_p]),
     "hbl_forward": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_size_t, _c_float, _c_int, _c_int, _c_int,
                              _c_int, _c_int, _c_float, _c_float, _c_void_p, _c_size_t, _c_void_p, _c_int,
                              _c_void_p]),
@@ -173,6 +182,25 @@ def hbl_pack_weights(W, eps_w: float = 0.0, packed=None, workspace=None, stream=
     return packed, alpha.value
 
 
+def hbl_pack_weights_rotated_workspace(K: int, N: int) -> int:
+    return lib().hbl_pack_weights_rotated_workspace(K, N)
+
+
+def hbl_pack_weights_rotated(W, had_block: int = 0, eps_w: float = 0.0, packed=None, workspace=None, stream=None):
+    """Rotate each column of fp32 W [K, N] by the activations' Hadamard transform along K, then
+    ternarise. Returns (packed uint8 blob, alpha)."""
+    K, N = W.shape
+    if packed is None:
+        packed = _u8_empty(hbl_packed_weights_bytes(K, N), W.device)
+    if workspace is None:
+        workspace = _u8_empty(hbl_pack_weights_rotated_workspace(K, N), W.device)
+    alpha = _c_float(0.0)
+    _check(lib().hbl_pack_weights_rotated(_ptr(W), K, N, int(had_block), float(eps_w), _ptr(packed), packed.numel(),
+                                          ctypes.byref(alpha), _ptr(workspace), workspace.numel(),
+                                          _stream(stream, W)), "hbl_pack_weights_rotated")
+    return packed, alpha.value
+
+
 def hbl_pack_ternary(t, packed=None, stream=None):
     """Pack given ternary codes t [K, N] (int8 in {-1, 0, 1}). Returns the packed blob."""
     K, N = t.shape
@@ -227,4 +255,41 @@ def hbl_forward(X, packed, alpha: float, N: int, gain=None, had_block: int = 0, 
     _check(lib().hbl_forward(_ptr(X), _ptr(gain), _ptr(packed), packed.numel(), float(alpha), M, K, N, had_block,
                              quant, float(eps_norm), float(eps_q), _ptr(workspace), workspace.numel(), _ptr(Y),
                              out_dtype, _stream(stream, X)), "hbl_forward")
+    return Y
+
+
+def hbl_qkv_codes_bytes(M: int, H: int, D: int, bits: int) -> int:
+    return lib().hbl_qkv_codes_bytes(M, H, D, bits)
+
+
+def hbl_qkv_quant(X, H: int, D: int, bits: int = 3, pos=None, rope_theta: float = 10000.0, row_stride=None,
+                  codes=None, gamma=None, stream=None):
+    """RoPE (when `pos`, int32 [M], is given) then per-head unsigned absmax quantisation of bf16 X,
+    token rows of `row_stride` elements (default H*D) holding H heads of D features from the
+    row start. Returns (codes uint8 [M, H, D*bits/8], gamma fp32 [M, H])."""
+    import torch
+
+    M = X.shape[0]
+    if row_stride is None:
+        row_stride = H * D
+    if codes is None:
+        codes = torch.empty((M, H, D * bits // 8), dtype=torch.uint8, device=X.device)
+    if gamma is None:
+        gamma = torch.empty((M, H), dtype=torch.float32, device=X.device)
+    if not X.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    _check(lib().hbl_qkv_quant(X.data_ptr(), int(row_stride), _ptr(pos), float(rope_theta), M, H, D, bits,
+                               _ptr(codes), codes.numel(), _ptr(gamma), _stream(stream, X)), "hbl_qkv_quant")
+    return codes, gamma
+
+
+def hbl_qkv_dequant(codes, gamma, D: int, bits: int, Y=None, stream=None):
+    """bf16 [M, H, D] from codes and gamma written by hbl_qkv_quant."""
+    import torch
+
+    M, H = gamma.shape
+    if Y is None:
+        Y = torch.empty((M, H, D), dtype=torch.bfloat16, device=codes.device)
+    _check(lib().hbl_qkv_dequant(_ptr(codes), _ptr(gamma), M, H, D, bits, _ptr(Y), _stream(stream, codes)),
+           "hbl_qkv_dequant")
     return Y

@@ -17,7 +17,9 @@
 #include "gemm_swap.cuh"
 #include "norm_fht_quant.cuh"
 #include "norm_fht_quant_tc.cuh"
+#include "norm_quant.cuh"
 #include "pack_weights.cuh"
+#include "qkv_quant.cuh"
 
 using namespace hbl;
 
@@ -179,8 +181,63 @@ hbl_status launch_nfq_tc(const NfqArgs& a, cudaStream_t s) {
   return HBL_OK;
 }
 
+// No transform (blocks of one feature): up to E features per thread, tpr threads per row (a
+// multiple of 32, at most 1024, tpr * E >= K), and at least 256 threads per CTA.
+template <int E>
+hbl_status launch_nq_e(const NqArgs& a0, int quant, cudaStream_t s) {
+  NqArgs a = a0;
+  const int vpt = E / 8;                                 // 16-byte vectors per thread
+  a.tpr = ((a.K / 8 + vpt - 1) / vpt + 31) / 32 * 32;   // K / 8 is a multiple of 32
+  a.rows = a.tpr >= 256 ? 1 : 256 / a.tpr;
+  auto pick = [&](auto k) -> hbl_status {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((a.M + a.rows - 1) / a.rows, 1, 1);
+    cfg.blockDim = dim3(a.tpr * a.rows, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may overlap the kernel before
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, k, a);
+    if (e != cudaSuccess) return cuda_fail(e);
+    HBL_CHECK_LAUNCH();
+    return HBL_OK;
+  };
+  if (a.gain) {
+    if (quant == 0) return pick(norm_quant_kernel<E, 0, true>);
+    if (quant == 1) return pick(norm_quant_kernel<E, 1, true>);
+    return pick(norm_quant_kernel<E, 2, true>);
+  }
+  if (quant == 0) return pick(norm_quant_kernel<E, 0, false>);
+  if (quant == 1) return pick(norm_quant_kernel<E, 1, false>);
+  return pick(norm_quant_kernel<E, 2, false>);
+}
+
+hbl_status run_nq(const void* X, const float* gain, int M, int K, int quant, float eps_norm, float eps_q, int fmt,
+                  void* codes, float* s_x, cudaStream_t stream) {
+  NqArgs a;
+  a.X = static_cast<const uint16_t*>(X);
+  a.gain = gain;
+  a.codes = static_cast<uint8_t*>(codes);
+  a.s_x = s_x;
+  a.M = M;
+  a.K = K;
+  a.fmt = fmt;
+  a.eps_norm = eps_norm;
+  a.eps_q = eps_q;
+  a.tpr = 0;
+  a.rows = 0;
+  // K is a multiple of 256 in [256, 32768], so tpr lands in [32, 1024]
+  if (K <= 2048) return launch_nq_e<8>(a, quant, stream);
+  if (K <= 16384) return launch_nq_e<16>(a, quant, stream);
+  return launch_nq_e<32>(a, quant, stream);
+}
+
 hbl_status run_nfq(const void* X, const float* gain, int M, int K, int had_block, int quant, float eps_norm,
                    float eps_q, int fmt, void* codes, float* s_x, cudaStream_t stream) {
+  if (had_block == 1) return run_nq(X, gain, M, K, quant, eps_norm, eps_q, fmt, codes, s_x, stream);
   const int n = had_block == 0 ? K : had_block;
   if (!is_pow2(n) || n < 256 || n > 16384 || (K % n) != 0) return HBL_EUNSUPPORTED;
   const int L = ilog2_c(n);
@@ -490,6 +547,85 @@ hbl_status run_gemm(const void* codes, int fmt, int abits, const float* s_x, con
   return run_tc2(codes, reinterpret_cast<const int8_t*>(blob + bl.off1), t, s);
 }
 
+// Ternarise fp32 W [K][N] into the packed blob (validated arguments): alpha reduced on the
+// device, codes packed, alpha read back (synchronises the stream).
+hbl_status pack_from_f32(const float* W, int K, int N, float eps_w, void* packed, float* alpha_host, void* workspace,
+                         cudaStream_t s) {
+  const BlobLayout bl = blob_layout(K, N);
+  uint8_t* blob = static_cast<uint8_t*>(packed);
+  double* partials = static_cast<double*>(workspace);
+  double* alpha_d = partials + kAbsumBlocks;
+  cudaError_t e = cudaMemsetAsync(blob + bl.off2, 0, (size_t)N * 4, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const size_t count = (size_t)K * N;
+  absum_partial_kernel<<<kAbsumBlocks, kAbsumThreads, 0, s>>>(W, count / 4, partials);
+  HBL_CHECK_LAUNCH();
+  absum_final_kernel<<<1, kAbsumThreads, 0, s>>>(partials, kAbsumBlocks, (double)count, alpha_d);
+  HBL_CHECK_LAUNCH();
+  dim3 grid((N + 127) / 128, K / 16);
+  ternarize_pack_kernel<false><<<grid, 128, 0, s>>>(W, nullptr, K, N, alpha_d, (double)eps_w,
+                                                     reinterpret_cast<uint32_t*>(blob + bl.off0),
+                                                     reinterpret_cast<int8_t*>(blob + bl.off1),
+                                                     reinterpret_cast<int32_t*>(blob + bl.off2));
+  HBL_CHECK_LAUNCH();
+  double alpha = 0.0;
+  e = cudaMemcpyAsync(&alpha, alpha_d, sizeof(double), cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  *alpha_host = (float)alpha;
+  return HBL_OK;
+}
+
+template <int E, int BITS>
+hbl_status launch_qkv(const QkvArgs& a, cudaStream_t s) {
+  const int warps = a.H < 8 ? a.H : 8;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.M, 1, 1);
+  cfg.blockDim = dim3(32 * warps, 1, 1);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may overlap the kernel before
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = a.pos ? cudaLaunchKernelEx(&cfg, qkv_quant_kernel<E, BITS, true>, a)
+                              : cudaLaunchKernelEx(&cfg, qkv_quant_kernel<E, BITS, false>, a);
+  if (e != cudaSuccess) return cuda_fail(e);
+  HBL_CHECK_LAUNCH();
+  return HBL_OK;
+}
+
+template <int E>
+hbl_status launch_qkv_e(const QkvArgs& a, int bits, cudaStream_t s) {
+  switch (bits) {
+    case 2: return launch_qkv<E, 2>(a, s);
+    case 3: return launch_qkv<E, 3>(a, s);
+    case 4: return launch_qkv<E, 4>(a, s);
+    default: return launch_qkv<E, 8>(a, s);
+  }
+}
+
+template <int E>
+hbl_status launch_qkv_dequant_e(const uint8_t* codes, const float* gamma, int M, int H, int bits, uint16_t* Y,
+                                cudaStream_t s) {
+  const size_t heads = (size_t)M * H;
+  const dim3 grid((unsigned)((heads + 7) / 8));
+  switch (bits) {
+    case 2: qkv_dequant_kernel<E, 2><<<grid, 256, 0, s>>>(codes, gamma, M, H, Y); break;
+    case 3: qkv_dequant_kernel<E, 3><<<grid, 256, 0, s>>>(codes, gamma, M, H, Y); break;
+    case 4: qkv_dequant_kernel<E, 4><<<grid, 256, 0, s>>>(codes, gamma, M, H, Y); break;
+    default: qkv_dequant_kernel<E, 8><<<grid, 256, 0, s>>>(codes, gamma, M, H, Y); break;
+  }
+  HBL_CHECK_LAUNCH();
+  return HBL_OK;
+}
+
+bool qkv_shape_ok(int M, int H, int D, int bits) {
+  return M >= 1 && H >= 1 && (D == 64 || D == 128 || D == 256) &&
+         (bits == 2 || bits == 3 || bits == 4 || bits == 8) && (size_t)M * H < ((size_t)1 << 36);
+}
+
 size_t forward_codes_bytes(int M, int K) { return round_up((size_t)M * K, 256); }
 
 }  // namespace
@@ -555,32 +691,55 @@ hbl_status hbl_pack_weights(const float* W, int K, int N, float eps_w, void* pac
   if (K < 256 || K > 32768 || (K % 256) || N < 1 || (N % 8)) return HBL_EINVAL;
   if (!aligned(W, 16) || !aligned(packed, 256) || !aligned(workspace, 16)) return HBL_EINVAL;
   if (!(eps_w >= 0.f)) return HBL_EINVAL;
-  const BlobLayout bl = blob_layout(K, N);
-  if (packed_bytes < bl.total || ws_bytes < hbl_pack_weights_workspace(K, N)) return HBL_EINVAL;
+  if (packed_bytes < blob_layout(K, N).total || ws_bytes < hbl_pack_weights_workspace(K, N)) return HBL_EINVAL;
+  return pack_from_f32(W, K, N, eps_w, packed, alpha_host, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t hbl_pack_weights_rotated_workspace(int K, int N) {
+  if (K <= 0 || N <= 0) return 0;
+  return round_up((size_t)K * N * 4, 256) + hbl_pack_weights_workspace(K, N);
+}
+
+hbl_status hbl_pack_weights_rotated(const float* W, int K, int N, int had_block, float eps_w, void* packed,
+                                    size_t packed_bytes, float* alpha_host, void* workspace, size_t ws_bytes,
+                                    hbl_stream_t stream) {
+  if (!W || !packed || !alpha_host || !workspace) return HBL_EINVAL;
+  if (K < 256 || K > 32768 || (K % 256) || N < 1 || (N % 8)) return HBL_EINVAL;
+  if (!aligned(W, 16) || !aligned(packed, 256) || !aligned(workspace, 256)) return HBL_EINVAL;
+  if (!(eps_w >= 0.f) || had_block < 0) return HBL_EINVAL;
+  if (packed_bytes < blob_layout(K, N).total || ws_bytes < hbl_pack_weights_rotated_workspace(K, N))
+    return HBL_EINVAL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  uint8_t* blob = static_cast<uint8_t*>(packed);
-  double* partials = static_cast<double*>(workspace);
-  double* alpha_d = partials + kAbsumBlocks;
-  cudaError_t e = cudaMemsetAsync(blob + bl.off2, 0, (size_t)N * 4, s);
-  if (e != cudaSuccess) return cuda_fail(e);
-  const size_t count = (size_t)K * N;
-  absum_partial_kernel<<<kAbsumBlocks, kAbsumThreads, 0, s>>>(W, count / 4, partials);
-  HBL_CHECK_LAUNCH();
-  absum_final_kernel<<<1, kAbsumThreads, 0, s>>>(partials, kAbsumBlocks, (double)count, alpha_d);
-  HBL_CHECK_LAUNCH();
-  dim3 grid((N + 127) / 128, K / 16);
-  ternarize_pack_kernel<false><<<grid, 128, 0, s>>>(W, nullptr, K, N, alpha_d, (double)eps_w,
-                                                     reinterpret_cast<uint32_t*>(blob + bl.off0),
-                                                     reinterpret_cast<int8_t*>(blob + bl.off1),
-                                                     reinterpret_cast<int32_t*>(blob + bl.off2));
-  HBL_CHECK_LAUNCH();
-  double alpha = 0.0;
-  e = cudaMemcpyAsync(&alpha, alpha_d, sizeof(double), cudaMemcpyDeviceToHost, s);
-  if (e != cudaSuccess) return cuda_fail(e);
-  e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) return cuda_fail(e);
-  *alpha_host = (float)alpha;
-  return HBL_OK;
+  if (had_block == 1)  // blocks of one feature: no rotation
+    return pack_from_f32(W, K, N, eps_w, packed, alpha_host, static_cast<uint8_t*>(workspace) +
+                         round_up((size_t)K * N * 4, 256), s);
+  const int n = had_block == 0 ? K : had_block;
+  if (!is_pow2(n) || n < 256 || n > 16384 || (K % n) != 0) return HBL_EUNSUPPORTED;
+  float* Wr = static_cast<float*>(workspace);
+  // the transform's log2(n) index bits in passes of at most 7 bits (2^7 rows x 32 columns of
+  // shared memory per CTA); the last pass applies 1/sqrt(n)
+  const int L = ilog2_c(n);
+  const int passes = (L + 6) / 7;
+  int b0 = 0;
+  for (int pi = 0; pi < passes; ++pi) {
+    const int nb = (L - b0) / (passes - pi);
+    const float scale = pi == passes - 1 ? (float)(1.0 / sqrt((double)n)) : 1.f;
+    const dim3 grid((N + 31) / 32, K >> nb);
+    const float* src = pi == 0 ? W : Wr;
+    switch (nb) {
+      case 1: fht_cols_kernel<1><<<grid, 256, 0, s>>>(src, Wr, K, N, b0, scale); break;
+      case 2: fht_cols_kernel<2><<<grid, 256, 0, s>>>(src, Wr, K, N, b0, scale); break;
+      case 3: fht_cols_kernel<3><<<grid, 256, 0, s>>>(src, Wr, K, N, b0, scale); break;
+      case 4: fht_cols_kernel<4><<<grid, 256, 0, s>>>(src, Wr, K, N, b0, scale); break;
+      case 5: fht_cols_kernel<5><<<grid, 256, 0, s>>>(src, Wr, K, N, b0, scale); break;
+      case 6: fht_cols_kernel<6><<<grid, 256, 0, s>>>(src, Wr, K, N, b0, scale); break;
+      default: fht_cols_kernel<7><<<grid, 256, 0, s>>>(src, Wr, K, N, b0, scale); break;
+    }
+    HBL_CHECK_LAUNCH();
+    b0 += nb;
+  }
+  return pack_from_f32(Wr, K, N, eps_w, packed, alpha_host,
+                       static_cast<uint8_t*>(workspace) + round_up((size_t)K * N * 4, 256), s);
 }
 
 hbl_status hbl_pack_ternary(const int8_t* t, int K, int N, void* packed, size_t packed_bytes,
@@ -632,6 +791,49 @@ hbl_status hbl_ternary_gemm(const void* codes, hbl_codes_fmt fmt, int abits, con
   if (packed_bytes < blob_layout(K, N).total) return HBL_EINVAL;
   return run_gemm(codes, (int)fmt, abits, s_x, packed, alpha, M, N, K, Y, (int)out_dtype, acc_debug,
                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t hbl_qkv_codes_bytes(int M, int H, int D, int bits) {
+  if (M <= 0 || H <= 0 || D <= 0 || bits <= 0) return 0;
+  return (size_t)M * H * D * bits / 8;
+}
+
+hbl_status hbl_qkv_quant(const void* X, size_t row_stride, const int32_t* pos, float rope_theta, int M, int H, int D,
+                         int bits, void* codes, size_t codes_bytes, float* gamma, hbl_stream_t stream) {
+  if (!X || !codes || !gamma) return HBL_EINVAL;
+  if (M < 1 || H < 1 || D < 1 || bits < 1) return HBL_EINVAL;
+  if (!qkv_shape_ok(M, H, D, bits)) return HBL_EUNSUPPORTED;
+  if (row_stride < (size_t)H * D || (row_stride % 8) != 0) return HBL_EINVAL;
+  if (!aligned(X, 16) || !aligned(codes, 16) || !aligned(gamma, 4) || (pos && !aligned(pos, 4))) return HBL_EINVAL;
+  if (pos && !(rope_theta > 1.f && rope_theta < 3.0e38f)) return HBL_EINVAL;
+  if (codes_bytes < hbl_qkv_codes_bytes(M, H, D, bits)) return HBL_EINVAL;
+  QkvArgs a;
+  a.X = static_cast<const uint16_t*>(X);
+  a.row_stride = row_stride;
+  a.pos = pos;
+  a.theta = rope_theta;
+  a.codes = static_cast<uint8_t*>(codes);
+  a.gamma = gamma;
+  a.M = M;
+  a.H = H;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (D == 64) return launch_qkv_e<2>(a, bits, s);
+  if (D == 128) return launch_qkv_e<4>(a, bits, s);
+  return launch_qkv_e<8>(a, bits, s);
+}
+
+hbl_status hbl_qkv_dequant(const void* codes, const float* gamma, int M, int H, int D, int bits, void* Y,
+                           hbl_stream_t stream) {
+  if (!codes || !gamma || !Y) return HBL_EINVAL;
+  if (M < 1 || H < 1 || D < 1 || bits < 1) return HBL_EINVAL;
+  if (!qkv_shape_ok(M, H, D, bits)) return HBL_EUNSUPPORTED;
+  if (!aligned(codes, 16) || !aligned(gamma, 4) || !aligned(Y, 16)) return HBL_EINVAL;
+  const uint8_t* c = static_cast<const uint8_t*>(codes);
+  uint16_t* y = static_cast<uint16_t*>(Y);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (D == 64) return launch_qkv_dequant_e<2>(c, gamma, M, H, bits, y, s);
+  if (D == 128) return launch_qkv_dequant_e<4>(c, gamma, M, H, bits, y, s);
+  return launch_qkv_dequant_e<8>(c, gamma, M, H, bits, y, s);
 }
 
 size_t hbl_forward_workspace(int M, int K, hbl_quant quant) {

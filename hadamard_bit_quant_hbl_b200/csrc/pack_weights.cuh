@@ -118,4 +118,43 @@ __global__ void __launch_bounds__(128) ternarize_pack_kernel(const float* __rest
   atomicAdd(sec2 + n, colsum);
 }
 
+// ---------------------------------------------------------------- weight-side rotation
+
+// One pass of the orthonormal Walsh-Hadamard transform along k, over index bits [b0, b0 + NB),
+// of every column of a row-major fp32 matrix [K][N] (the variant with rotated weights and
+// activations of the walkthrough article's Table 5 ablation: W' = H W along the reduction
+// dimension, before ternarisation). A CTA holds the 2^NB rows k = hi * 2^(b0+NB) + j * 2^b0 + lo
+// (j = 0 .. 2^NB - 1; hi, lo fixed per CTA) of 32 consecutive columns in shared memory, runs the
+// NB butterfly stages (a, b) -> (a + b, a - b) of pairs j, j + h, and writes the rows back times
+// `scale`. Every CTA reads and writes only its own elements, so src may equal dst. K must be a
+// multiple of 2^(b0+NB).
+template <int NB>
+__global__ void __launch_bounds__(256) fht_cols_kernel(const float* src, float* dst, int K, int N, int b0,
+                                                       float scale) {
+  constexpr int R = 1 << NB;
+  __shared__ float tile[R][33];
+  const int c = threadIdx.x & 31;
+  const int col = blockIdx.x * 32 + c;
+  const bool live = col < N;
+  const size_t g = blockIdx.y;
+  const size_t lo = g & ((1u << b0) - 1u), hi = g >> b0;
+  const size_t kbase = (hi << (b0 + NB)) + lo;
+  for (int j = threadIdx.x >> 5; j < R; j += 8)
+    tile[j][c] = live ? src[(kbase + ((size_t)j << b0)) * (size_t)N + col] : 0.f;
+  __syncthreads();
+#pragma unroll
+  for (int h = 1; h < R; h <<= 1) {
+    for (int p = threadIdx.x; p < (R / 2) * 32; p += 256) {
+      const int cc = p & 31, bi = p >> 5;
+      const int j0 = (bi / h) * 2 * h + (bi % h);
+      const float a = tile[j0][cc], b = tile[j0 + h][cc];
+      tile[j0][cc] = a + b;
+      tile[j0 + h][cc] = a - b;
+    }
+    __syncthreads();
+  }
+  if (!live) return;
+  for (int j = threadIdx.x >> 5; j < R; j += 8) dst[(kbase + ((size_t)j << b0)) * (size_t)N + col] = tile[j][c] * scale;
+}
+
 }  // namespace hbl

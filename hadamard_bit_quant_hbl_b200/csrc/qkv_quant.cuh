@@ -1,0 +1,165 @@
+// QKV states after RoPE, quantised per head to unsigned b-bit integers with an absmax scale (the
+// low-bit attention states and 3-bit KV cache of BitNet v2), and the matching dequantisation.
+//
+// Method: BitNet v2 walkthrough article (m.jxzklqfsx.com), section "實驗結果" (Tables 2-3): the
+// QKV states are quantised after RoPE; each head goes directly to unsigned integers through the
+// absmax function, with no calibration data. The formulas were not preserved, so this follows the
+// plainest reading: per token and head, gamma = max|x| over the head's D features, and
+// [-gamma, gamma] maps linearly onto [0, 2^b - 1]:
+//     u = RoundClip((2^b - 1)/2 * (x/gamma + 1), 0, 2^b - 1),   x~ = (2u - (2^b - 1)) gamma/(2^b - 1).
+// RoPE is the LLaMA form of the model's LLaMA-like parts ("BitNet v2：原生4位激活"): feature f of a
+// head pairs with f + D/2 and both turn by the angle pos * theta^(-2f/D).
+//
+// Layout: one CTA per token. Its threads first build the cos/sin table of the token's D/2 angles
+// in shared memory (angle formed and reduced modulo 2 pi in fp64, then rounded to fp32), then each
+// warp takes heads in turn: lane l holds features l*E .. l*E+E-1 (E = D/32), whose RoPE partners
+// sit in lane l ^ 16. Codes leave as a little-endian bit string per head (code j at bits
+// [b j, b j + b)), each group of 8 codes (b bytes) assembled across the lanes that hold it.
+#pragma once
+
+#include "common.cuh"
+
+namespace hbl {
+
+struct QkvArgs {
+  const uint16_t* X;  // bf16; token m, head h at X + m * row_stride + h * D
+  size_t row_stride;  // elements between consecutive tokens
+  const int32_t* pos; // [M] token positions, or nullptr: no RoPE (the V states)
+  float theta;
+  uint8_t* codes;     // [M][H][D * bits / 8]
+  float* gamma;       // [M][H]
+  int M, H;
+};
+
+template <int E>
+__device__ __forceinline__ void qkv_load(const uint16_t* p, float (&v)[E]) {
+  if constexpr (E == 2) {
+    const uint32_t u = __ldg(reinterpret_cast<const unsigned int*>(p));
+    v[0] = __uint_as_float(u << 16);
+    v[1] = __uint_as_float(u & 0xffff0000u);
+  } else if constexpr (E == 4) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    v[0] = __uint_as_float(u.x << 16);
+    v[1] = __uint_as_float(u.x & 0xffff0000u);
+    v[2] = __uint_as_float(u.y << 16);
+    v[3] = __uint_as_float(u.y & 0xffff0000u);
+  } else {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+}
+
+// Stores the GB bytes of a code group (GB = bits) at p.
+template <int GB>
+__device__ __forceinline__ void qkv_store_group(uint8_t* p, uint64_t g) {
+  if constexpr (GB == 8) {
+    *reinterpret_cast<uint2*>(p) = make_uint2((uint32_t)g, (uint32_t)(g >> 32));
+  } else if constexpr (GB == 4) {
+    *reinterpret_cast<uint32_t*>(p) = (uint32_t)g;
+  } else if constexpr (GB == 2) {
+    *reinterpret_cast<uint16_t*>(p) = (uint16_t)g;
+  } else {
+#pragma unroll
+    for (int i = 0; i < GB; ++i) p[i] = (uint8_t)(g >> (8 * i));
+  }
+}
+
+template <int E, int BITS, bool ROPE>
+__global__ void __launch_bounds__(256) qkv_quant_kernel(QkvArgs a) {
+  static_assert(E == 2 || E == 4 || E == 8, "head size 64, 128 or 256");
+  constexpr int D = 32 * E, HALF = D / 2;
+  constexpr float kL = (float)((1 << BITS) - 1);
+  constexpr int LPG = 8 / E;  // lanes holding one group of 8 codes
+  constexpr int HEAD_BYTES = D * BITS / 8;
+  __shared__ float cs[HALF], sn[HALF];
+
+  const int m = blockIdx.x;
+  // X may come from the kernel before this one (programmatic dependent launch)
+  pdl_wait();
+  pdl_launch_dependents();
+  if constexpr (ROPE) {
+    const double two_pi = 6.283185307179586476925;
+    const double lt = log((double)a.theta);
+    const double p = (double)a.pos[m];
+    for (int f = threadIdx.x; f < HALF; f += blockDim.x) {
+      const double ang = p * exp(-2.0 * (double)f / (double)D * lt);
+      const double r = ang - two_pi * rint(ang / two_pi);
+      double s, c;
+      sincos(r, &s, &c);
+      cs[f] = (float)c;
+      sn[f] = (float)s;
+    }
+    __syncthreads();
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const uint16_t* xrow = a.X + (size_t)m * a.row_stride;
+  for (int h = warp; h < a.H; h += nwarps) {
+    float v[E];
+    qkv_load<E>(xrow + (size_t)h * D + lane * E, v);
+    if constexpr (ROPE) {
+      const bool first = lane < 16;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float partner = __shfl_xor_sync(0xffffffffu, v[e], 16);
+        const int f = (lane & 15) * E + e;
+        const float c = cs[f], s = sn[f];
+        v[e] = first ? fmaf(v[e], c, -partner * s) : fmaf(partner, s, v[e] * c);
+      }
+    }
+    float g = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) g = fmaxf(g, fabsf(v[e]));
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, o));
+    const float mult = g > 0.f ? 0.5f * kL / g : 0.f;
+    unsigned long long bits = 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float q = fminf(fmaxf(rintf(fmaf(v[e], mult, 0.5f * kL)), 0.f), kL);
+      bits |= (unsigned long long)(uint32_t)q << (((lane % LPG) * E + e) * BITS);
+    }
+#pragma unroll
+    for (int o = 1; o < LPG; o <<= 1) bits |= __shfl_xor_sync(0xffffffffu, bits, o);
+    const size_t mh = (size_t)m * a.H + h;
+    if (lane % LPG == 0) qkv_store_group<BITS>(a.codes + mh * HEAD_BYTES + (lane / LPG) * BITS, bits);
+    if (lane == 0) a.gamma[mh] = g;
+  }
+}
+
+// x~ = (2u - (2^b - 1)) * gamma / (2^b - 1) as bf16 [M][H][D]: one warp per head, lane l
+// producing features l*E .. l*E+E-1.
+template <int E, int BITS>
+__global__ void __launch_bounds__(256) qkv_dequant_kernel(const uint8_t* __restrict__ codes,
+                                                          const float* __restrict__ gamma, int M, int H,
+                                                          uint16_t* __restrict__ Y) {
+  constexpr int D = 32 * E;
+  constexpr int HEAD_BYTES = D * BITS / 8;
+  constexpr float kL = (float)((1 << BITS) - 1);
+  const int lane = threadIdx.x & 31;
+  const size_t mh = (size_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (mh >= (size_t)M * H) return;
+  const uint8_t* hp = codes + mh * HEAD_BYTES;
+  const int b0 = lane * E * BITS;
+  const int byte0 = b0 >> 3, shift = b0 & 7;
+  const int nbytes = (shift + E * BITS + 7) >> 3;
+  uint64_t w = 0;
+  for (int i = 0; i < nbytes; ++i) w |= (uint64_t)hp[byte0 + i] << (8 * i);
+  w >>= shift;
+  const float step = gamma[mh] / kL;
+  uint16_t* out = Y + mh * D + lane * E;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const float u = (float)((w >> (e * BITS)) & ((1u << BITS) - 1u));
+    const float x = (2.f * u - kL) * step;
+    // round to nearest even bf16
+    const uint32_t xb = __float_as_uint(x);
+    out[e] = (uint16_t)((xb + 0x7fffu + ((xb >> 16) & 1u)) >> 16);
+  }
+}
+
+}  // namespace hbl

@@ -36,6 +36,7 @@ __all__ = [
     "activations",
     "weights",
     "layer",
+    "qkv_states",
 ]
 
 
@@ -62,7 +63,7 @@ class LayerSpec:
     K: int
     N: int
     abits: int
-    had_block: int  # 0 = one transform over all of K (K a power of two); else block size
+    had_block: int  # 0 = one transform over all of K (K a power of two); 1 = none; else block size
     dist: str  # "normal" or "laplace"
     scale: float  # std (normal) or diversity b (laplace) of the body
     zero_frac: float  # fraction of body values set to exactly 0
@@ -85,8 +86,9 @@ class LayerSpec:
         )
 
 
-# The five workload families. Sizes follow the 1.3B / 3B / 7B-like Wo and Wdown shapes.
-# The 7B pair is listed at its largest token count; other token counts use with_m().
+# The five H-BitLinear workload families (sizes follow the 1.3B / 3B / 7B-like Wo and Wdown
+# shapes) and one plain BitLinear. The 7B pair is listed at its largest token count; other token
+# counts use with_m().
 WORKLOADS: dict[str, LayerSpec] = {
     "single_a8_16x256": LayerSpec(
         "single_a8_16x256", 16, 256, 256, 8, 0, "normal", 1.0, 0.0, 4 / 256, 50.0, 0,
@@ -106,6 +108,12 @@ WORKLOADS: dict[str, LayerSpec] = {
     "wdown_nonpow2_a4": LayerSpec(
         "wdown_nonpow2_a4", 8192, 11008, 4096, 4, 256, "laplace", 0.05, 0.0, 0.01, 50.0, 4,
         note="Wdown with K=11008 = 43 x 256, block-diagonal transform"),
+    # A plain BitLinear (no rotation, had_block = 1). The walkthrough article (section
+    # "H-BitLinear模塊") describes the inputs of the attention and FFN input projections as roughly
+    # Gaussian, unlike the outlier-heavy Wo/Wdown inputs: a normal body without outlier channels.
+    "qkv_7b_plain_a4": LayerSpec(
+        "qkv_7b_plain_a4", 8192, 4096, 12288, 4, 1, "normal", 1.0, 0.0, 0.0, 1.0, 5,
+        note="7B-like fused QKV projection 4096 -> 12288, no transform, N(0,1) inputs"),
 }
 
 # Token counts of the 7B-like layer pair sweep.
@@ -148,3 +156,16 @@ def layer(name: str, M: int | None = None) -> tuple[LayerSpec, np.ndarray, np.nd
     if M is not None:
         spec = spec.with_m(M)
     return spec, activations(spec), weights(spec)
+
+
+def qkv_states(M: int, H: int, D: int, seed: int = 6, row_stride: int | None = None) -> np.ndarray:
+    """bf16 bit patterns [M, row_stride] of attention states: M tokens of H heads x D features from
+    the row start, N(0, 1) (the pages give no distribution for the QKV states), drawn row by row
+    from numpy PCG64 seeded with [seed, H, D]; features past H*D (another projection's slice of a
+    fused QKV row) are N(0, 1) as well."""
+    stride = H * D if row_stride is None else row_stride
+    rng = np.random.default_rng([seed, H, D])
+    out = np.empty((M, stride), dtype=np.uint16)
+    for i in range(M):
+        out[i] = f32_to_bf16_bits(rng.standard_normal(stride, dtype=np.float32))
+    return out

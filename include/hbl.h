@@ -119,6 +119,27 @@ hbl_status hbl_pack_weights(const float* W, int K, int N, float eps_w, void* pac
                             size_t packed_bytes, float* alpha_host, void* workspace,
                             size_t ws_bytes, hbl_stream_t stream);
 
+/* ---------------------------------------------------------------------------------------
+ * Rotated weights: the variant of the walkthrough article's Table 5 ablation (section
+ * "與其他後訓練量化方法的對比") that applies the Hadamard rotation to the weights as well as to the
+ * activations. Each column of W (the K input weights of one output feature) is rotated by the
+ * same transform the activations get, W' = H W along K, and W' is ternarised as in
+ * hbl_pack_weights. Since H is orthonormal and symmetric, (H xhat)^T (H W) = xhat^T W: run
+ * hbl_forward with the same had_block to compute the layer in the rotated bases.
+ *   had_block  0 (one transform over all of K, a power of two in [256, 16384]), a power of two
+ *              in [256, 16384] dividing K (block-diagonal), or 1 (no rotation: the same result
+ *              as hbl_pack_weights)
+ *   workspace  device scratch of ws_bytes >= hbl_pack_weights_rotated_workspace(K, N), 256-byte
+ *              aligned (it receives W' in fp32, K*N*4 bytes, then the alpha partial sums)
+ *   other arguments as for hbl_pack_weights. HBL_EUNSUPPORTED for another had_block.
+ * The rotation runs in fp32 (log2(n) butterfly stages, then 1/sqrt(n)); alpha and the rounding
+ * decision are taken in fp64 on W'. Synchronises `stream` before returning. */
+size_t hbl_pack_weights_rotated_workspace(int K, int N);
+
+hbl_status hbl_pack_weights_rotated(const float* W, int K, int N, int had_block, float eps_w,
+                                    void* packed, size_t packed_bytes, float* alpha_host,
+                                    void* workspace, size_t ws_bytes, hbl_stream_t stream);
+
 /* Pack given ternary codes t [K][N] (int8 in {-1,0,1}, row-major) into `packed`.
  * Entries outside {-1,0,1} give HBL_EINVAL only through hbl_device_status (they are
  * clamped and flagged, not trapped). Asynchronous. */
@@ -139,13 +160,16 @@ hbl_status hbl_pack_ternary(const int8_t* t, int K, int N, void* packed, size_t 
  *            decide in fp32, so a value within fp32 rounding of a .5 boundary may land on
  *            either side of it (a one-step code difference from an exact evaluation).
  * Kernels: one block of 4096, 8192 or 16384 features without gain runs the H_128 Kronecker factor of
- * the transform on the tensor cores and the rest on CUDA cores; every other shape runs on CUDA
- * cores. Both give the same codes up to the rounding-order ties the parity tests allow.
+ * the transform on the tensor cores and the rest on CUDA cores; had_block = 1 runs a streaming
+ * norm-and-quantise kernel; every other shape runs the CUDA-core transform. Both give the same codes up to the rounding-order ties the parity tests allow.
  *
  *   X       device bf16 [M][K], 16-byte aligned
  *   gain    device fp32 [K] or NULL
  *   had_block 0, or a power of two in [256, 16384] dividing K; when 0, K must be a power of two
- *           in [256, 16384]
+ *           in [256, 16384]. had_block = 1 is the block-diagonal transform with blocks of one
+ *           feature (H_1 = [1]), i.e. no rotation: the plain BitLinear of every other linear
+ *           layer (QKV, up/gate), which the walkthrough article's section
+ *           "BitNet v2：原生4位激活" runs with the same INT4/INT8 activations
  *   codes   device, M rows in `fmt` (see hbl_codes_fmt), 16-byte aligned
  *   s_x     device fp32 [M]
  * Asynchronous. */
@@ -186,6 +210,42 @@ hbl_status hbl_forward(const void* X, const float* gain, const void* packed, siz
                        float alpha, int M, int K, int N, int had_block, hbl_quant quant,
                        float eps_norm, float eps_q, void* workspace, size_t ws_bytes, void* Y,
                        hbl_out_dtype out_dtype, hbl_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Low-bit attention states: QKV quantised after RoPE to unsigned integers per head.
+ *
+ * The walkthrough article (section "實驗結果", Tables 2-3) quantises the QKV states after RoPE,
+ * each head directly to unsigned integers with the absmax function and no calibration data, and
+ * reports that a 3-bit KV cache matches full precision. Its formulas were lost; this library
+ * reads them as follows, per token m and head h (D features):
+ *   RoPE (Q and K only; pos given): feature f < D/2 pairs with f + D/2, both turned by the angle
+ *        pos[m] * theta^(-2f/D):  (x_f, x_{f+D/2}) -> (x_f c - x_{f+D/2} s, x_f s + x_{f+D/2} c)
+ *   gamma[m][h] = max_d |x[d]|
+ *   u[d] = RoundClip((2^b - 1)/2 * (x[d]/gamma + 1), 0, 2^b - 1)   (a zero head: x/gamma = 0)
+ *   dequantised: x~[d] = (2 u[d] - (2^b - 1)) * gamma / (2^b - 1)
+ * Codes of a head form a little-endian bit string of D*b bits: code d at bits [b d, b d + b)
+ * (bit i of the string is bit i%8 of byte i/8); heads follow each other, [M][H][D*b/8] bytes.
+ *
+ *   X          device bf16; token m, head h starts at element m*row_stride + h*D; 16-byte aligned
+ *   row_stride elements between tokens, >= H*D and a multiple of 8 (so Q, K or V can be read in
+ *              place from a fused QKV output)
+ *   pos        device int32 [M] token positions, or NULL for no rotation (the V states)
+ *   rope_theta RoPE base (> 1; LLaMA uses 10000); ignored when pos is NULL
+ *   D          64, 128 or 256; bits 2, 3, 4 or 8 (else HBL_EUNSUPPORTED)
+ *   codes      device, codes_bytes >= hbl_qkv_codes_bytes(M, H, D, bits), 16-byte aligned
+ *   gamma      device fp32 [M][H]
+ * The angle is formed and reduced modulo 2 pi in fp64, its cosine and sine rounded to fp32; the
+ * rotation and the rounding decision run in fp32. Asynchronous. */
+size_t hbl_qkv_codes_bytes(int M, int H, int D, int bits);
+
+hbl_status hbl_qkv_quant(const void* X, size_t row_stride, const int32_t* pos, float rope_theta,
+                         int M, int H, int D, int bits, void* codes, size_t codes_bytes,
+                         float* gamma, hbl_stream_t stream);
+
+/* Dequantise codes written by hbl_qkv_quant into bf16 Y [M][H][D] (16-byte aligned), rounded to
+ * nearest even. Asynchronous. */
+hbl_status hbl_qkv_dequant(const void* codes, const float* gamma, int M, int H, int D, int bits,
+                           void* Y, hbl_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------
  * hbl_forward without a caller-provided workspace. This entry point has no counterpart in the

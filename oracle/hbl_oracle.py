@@ -37,11 +37,22 @@ Readings taken where the pages are silent or the formulas were dropped
      decision included, is taken in float64 on the float64 values of the steps
      before it: q = clip(rint(Q * x / (stat + eps)), lo, hi).
   R6 output: y[m, n] = s[m] * alpha * sum_k q[m, k] t[k, n], evaluated in float64.
+  R7 rotated weights (optional): W' = H W along K with the activations' transform,
+     then R1 on W'.
+  R8 RoPE on the Q and K states (LLaMA-like parts): the rotate-half form, frequency f of
+     a head of D features pairing features f and f + D/2 with the angle
+     pos * theta^(-2f/D); theta is a parameter (10000 by default).
+  R9 QKV quantisation after RoPE to unsigned b-bit integers with an absmax scale, per
+     token and head: gamma = max|x| over the head's D values, the interval
+     [-gamma, gamma] mapped linearly onto [0, 2^b - 1]:
+       u = RoundClip((2^b - 1)/2 * (x/gamma + 1), 0, 2^b - 1),
+       x~ = (2u - (2^b - 1)) * gamma / (2^b - 1);
+     a head whose gamma is 0 takes x/gamma = 0.
 
 Parity status: every function below names the tests that pin it against
 something other than itself (closed forms, a dense Sylvester matrix from
 SciPy, torch's bf16 widening, brute force on small inputs, a hand-derived
-worked example). The choice of readings R1-R6 themselves is not pinned by any
+worked example). The choice of readings R1-R7 themselves is not pinned by any
 number on the pages, which print none: against the published method the
 oracle is "parity unpinned" in that sense only.
 """
@@ -60,10 +71,15 @@ __all__ = [
     "fwht",
     "hadamard_transform",
     "quantize",
+    "rotate_weights",
     "norm_fht_quant",
     "ternary_matmul",
     "dequant",
     "h_bitlinear_forward",
+    "rope",
+    "quantize_unsigned_absmax",
+    "dequantize_unsigned",
+    "qkv_quant",
 ]
 
 
@@ -221,6 +237,22 @@ def norm_fht_quant(x: np.ndarray, gain: np.ndarray | None, had_block: int, abits
     return quantize(xr, abits, scale_mode, eps_q)
 
 
+def rotate_weights(W: np.ndarray, block: int = 0) -> np.ndarray:
+    """Weight-side Hadamard rotation, W' = H W along K (reading R7).
+
+    [ART] section "與其他後訓練量化方法的對比", Table 5: the Hadamard rotation applied to the
+    weights and the activations, or to the activations only, both stabilise low-bit training.
+    With rotated weights each column of W (the K weights of one output feature) goes through the
+    same transform as the activations, so that (H x)^T (H W) = x^T W in exact arithmetic.
+
+    Pinned by test_rotate_weights_undoes_a_rotation (W = H T c ternarises back to T with
+    alpha = c * mean|T|), test_rotate_weights_columns_closed_form (a unit column gives the Walsh
+    column) and test_rotated_layer_keeps_the_full_precision_product.
+    """
+    W = np.asarray(W, dtype=np.float64)
+    return hadamard_transform(W.T, block).T
+
+
 def ternary_matmul(q: np.ndarray, t: np.ndarray) -> np.ndarray:
     """acc[m, n] = sum_k q[m, k] * t[k, n] in exact int64 arithmetic (the sum written as an einsum).
 
@@ -239,14 +271,73 @@ def dequant(acc: np.ndarray, s: np.ndarray, alpha: float) -> np.ndarray:
 
 def h_bitlinear_forward(x: np.ndarray, W: np.ndarray, gain: np.ndarray | None = None,
                         had_block: int = 0, abits: int = 4, scale_mode: str | None = None,
-                        eps_norm: float = 1e-6, eps_q: float = 0.0, eps_w: float = 0.0) -> dict:
+                        eps_norm: float = 1e-6, eps_q: float = 0.0, eps_w: float = 0.0,
+                        rotate_w: bool = False) -> dict:
     """The whole layer: weights ternarised, activations normed/rotated/quantised, product, dequant.
 
+    had_block = 1 is the plain BitLinear (no rotation). rotate_w rotates the latent weights with
+    the same transform before ternarising them (reading R7).
     Returns a dict with every intermediate (t, alpha, q, s, acc, y) for parity checks.
     """
     if scale_mode is None:
         scale_mode = "absmax" if abits == 8 else "absmean"
-    t, alpha = absmean_ternarize(W, eps_w)
+    t, alpha = absmean_ternarize(rotate_weights(W, had_block) if rotate_w else W, eps_w)
     q, s = norm_fht_quant(x, gain, had_block, abits, scale_mode, eps_norm, eps_q)
     acc = ternary_matmul(q, t)
     return {"t": t, "alpha": alpha, "q": q, "s": s, "acc": acc, "y": dequant(acc, s, alpha)}
+
+
+def rope(x: np.ndarray, pos: np.ndarray, theta: float = 10000.0) -> np.ndarray:
+    """Rotary position embedding of x [M, H, D] at token positions pos [M] (reading R8).
+
+    [ART] section "實驗結果": the QKV states are quantised after RoPE (rotary position
+    embedding); the model is LLaMA-like ("BitNet v2：原生4位激活"), whose RoPE rotates the pair
+    of features (f, f + D/2) of every head by the angle pos * theta^(-2f/D).
+
+    Pinned by test_rope_identity_norm_and_inverse (position 0, pair norms, rotating back),
+    test_rope_one_hot_closed_form and test_rope_depends_on_relative_position.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    D = x.shape[-1]
+    half = D // 2
+    inv = np.float64(theta) ** (-2.0 * np.arange(half) / D)
+    ang = np.asarray(pos, dtype=np.float64)[:, None] * inv[None, :]
+    c = np.cos(ang)[:, None, :]
+    s = np.sin(ang)[:, None, :]
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x1 * s + x2 * c], axis=-1)
+
+
+def quantize_unsigned_absmax(x: np.ndarray, bits: int) -> tuple[np.ndarray, np.ndarray]:
+    """Per-head absmax quantisation to unsigned b-bit integers (reading R9).
+
+    [ART] section "實驗結果": the QKV heads are quantised directly to unsigned integers with
+    the absmax function, with no calibration set; a 3-bit KV cache matches full precision.
+    x: [..., D]. Returns (u uint8 [..., D], gamma float64 [...]).
+
+    Pinned by test_unsigned_quantiser_properties (range, extremes, half-step error bound,
+    brute-force nearest level) and test_unsigned_quantiser_closed_form.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    L = (1 << bits) - 1
+    g = np.abs(x).max(axis=-1)
+    r = np.where(g[..., None] > 0, x / np.where(g > 0, g, 1.0)[..., None], 0.0)
+    u = np.clip(np.rint(L / 2.0 * (r + 1.0)), 0, L).astype(np.uint8)
+    return u, g
+
+
+def dequantize_unsigned(u: np.ndarray, gamma: np.ndarray, bits: int) -> np.ndarray:
+    """x~ = (2u - (2^b - 1)) * gamma / (2^b - 1) (reading R9)."""
+    L = (1 << bits) - 1
+    return (2.0 * np.asarray(u, dtype=np.float64) - L) * np.asarray(gamma, dtype=np.float64)[..., None] / L
+
+
+def qkv_quant(x: np.ndarray, pos: np.ndarray | None, bits: int, theta: float = 10000.0
+              ) -> tuple[np.ndarray, np.ndarray]:
+    """RoPE (when pos is given: the Q and K states; V takes none) then per-head unsigned absmax
+    quantisation of x [M, H, D] (float64 values or bf16 bit patterns). Returns (u, gamma)."""
+    if x.dtype == np.uint16:
+        x = bf16_to_f64(x)
+    if pos is not None:
+        x = rope(x, pos, theta)
+    return quantize_unsigned_absmax(x, bits)

@@ -62,3 +62,14 @@ def row_rel_err(y: np.ndarray, ref: np.ndarray) -> np.ndarray:
     num = np.linalg.norm(np.asarray(y, np.float64) - ref, axis=1)
     den = np.linalg.norm(ref, axis=1)
     return np.where(den > 0, num / np.where(den > 0, den, 1), num)
+
+
+def unpack_bitstream(packed: np.ndarray, D: int, bits: int) -> np.ndarray:
+    """Codes of hbl_qkv_quant: [..., D*bits/8] bytes, code d at bits [bits*d, bits*d + bits) of the
+    little-endian bit string of each head -> uint8 [..., D]."""
+    p = np.asarray(packed, dtype=np.uint8)
+    lead = p.shape[:-1]
+    bitarr = np.unpackbits(p.reshape(-1, p.shape[-1]), axis=-1, bitorder="little")  # [n, D*bits]
+    bitarr = bitarr.reshape(-1, D, bits).astype(np.uint16)
+    vals = (bitarr << np.arange(bits, dtype=np.uint16)).sum(axis=-1)
+    return vals.astype(np.uint8).reshape(*lead, D)

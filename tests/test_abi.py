@@ -119,3 +119,32 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(hbl, "library_path", str(tmp_path / "nope.so"))
     with pytest.raises(ImportError):
         hbl.lib()
+
+
+def test_pack_weights_rotated_rejects_bad_arguments(L):
+    f = hbl.lib().hbl_pack_weights_rotated
+    alpha = ctypes.c_float(0.0)
+    ws = hbl.hbl_pack_weights_rotated_workspace(4096, 64)
+    assert ws >= 4096 * 64 * 4
+    # NULL pointers, a bad K, a negative or unsupported block: refused on the host
+    assert f(None, 4096, 64, 0, 0.0, None, 0, ctypes.byref(alpha), None, 0, None) == hbl.HBL_EINVAL
+    assert f(FAKE, 4000, 64, 0, 0.0, FAKE, 1 << 30, ctypes.byref(alpha), FAKE, 1 << 30, None) == hbl.HBL_EINVAL
+    assert f(FAKE, 4096, 64, -1, 0.0, FAKE, 1 << 30, ctypes.byref(alpha), FAKE, 1 << 30, None) == hbl.HBL_EINVAL
+    assert f(FAKE, 4096, 64, 0, 0.0, FAKE, 1 << 30, ctypes.byref(alpha), FAKE, 16, None) == hbl.HBL_EINVAL
+    assert f(FAKE, 4096, 64, 96, 0.0, FAKE, 1 << 30, ctypes.byref(alpha), FAKE, 1 << 30, None) == hbl.HBL_EUNSUPPORTED
+
+
+def test_qkv_quant_rejects_bad_arguments(L):
+    f = hbl.lib().hbl_qkv_quant
+    big = 1 << 30
+    assert hbl.hbl_qkv_codes_bytes(10, 4, 128, 3) == 10 * 4 * 48
+    assert f(None, 512, None, 10000.0, 1, 4, 128, 3, FAKE, big, FAKE, None) == hbl.HBL_EINVAL
+    assert f(FAKE, 512, None, 10000.0, 1, 4, 96, 3, FAKE, big, FAKE, None) == hbl.HBL_EUNSUPPORTED
+    assert f(FAKE, 512, None, 10000.0, 1, 4, 128, 5, FAKE, big, FAKE, None) == hbl.HBL_EUNSUPPORTED
+    assert f(FAKE, 500, None, 10000.0, 1, 4, 128, 3, FAKE, big, FAKE, None) == hbl.HBL_EINVAL  # stride < H*D
+    assert f(FAKE, 516, None, 10000.0, 1, 4, 128, 3, FAKE, big, FAKE, None) == hbl.HBL_EINVAL  # stride % 8
+    assert f(FAKE, 512, FAKE, 0.5, 1, 4, 128, 3, FAKE, big, FAKE, None) == hbl.HBL_EINVAL      # theta
+    assert f(FAKE, 512, None, 10000.0, 1, 4, 128, 3, FAKE, 100, FAKE, None) == hbl.HBL_EINVAL  # codes too small
+    d = hbl.lib().hbl_qkv_dequant
+    assert d(None, FAKE, 1, 4, 128, 3, FAKE, None) == hbl.HBL_EINVAL
+    assert d(FAKE, FAKE, 1, 4, 100, 3, FAKE, None) == hbl.HBL_EUNSUPPORTED

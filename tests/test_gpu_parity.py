@@ -112,6 +112,51 @@ def test_norm_fht_quant_matches_oracle(K, had_block, M, quant, fmt, use_gain):
     np.testing.assert_allclose(s, s_ref, rtol=1e-5)
 
 
+# plain BitLinear (had_block = 1: blocks of one feature, no rotation), the other linears' inputs
+NQ_CASES = [
+    (256, 16, hbl.HBL_Q_A8_ABSMAX, hbl.HBL_CODES_PACKED, False),
+    (768, 37, hbl.HBL_Q_A4_ABSMEAN, hbl.HBL_CODES_PACKED, True),
+    (2304, 9, hbl.HBL_Q_A4_ABSMAX, hbl.HBL_CODES_I8, False),
+    (4096, 300, hbl.HBL_Q_A4_ABSMEAN, hbl.HBL_CODES_I8, False),
+    (4096, 5, hbl.HBL_Q_A8_ABSMAX, hbl.HBL_CODES_I8, True),
+    (8448, 7, hbl.HBL_Q_A4_ABSMEAN, hbl.HBL_CODES_PACKED, False),
+    (11008, 33, hbl.HBL_Q_A4_ABSMEAN, hbl.HBL_CODES_I8, True),
+    (16384, 3, hbl.HBL_Q_A4_ABSMAX, hbl.HBL_CODES_PACKED, False),
+    (17152, 2, hbl.HBL_Q_A4_ABSMEAN, hbl.HBL_CODES_I8, False),
+    (32768, 4, hbl.HBL_Q_A8_ABSMAX, hbl.HBL_CODES_I8, True),
+]
+
+
+@pytest.mark.parametrize("K,M,quant,fmt,use_gain", NQ_CASES)
+def test_norm_quant_without_transform_matches_oracle(K, M, quant, fmt, use_gain):
+    spec = spec_like("wo_7b_a4", K=K, M=M, seed=7 + K)
+    x = inputs.activations(spec)
+    gain = np.random.default_rng(K + 1).uniform(0.5, 1.5, size=K).astype(np.float32) if use_gain else None
+    abits, mode = QUANT_NAME[quant]
+    q_ref, s_ref = oracle.norm_fht_quant(x, gain, 1, abits, mode)
+    q, s = gpu_codes(x, gain, 1, quant, fmt)
+    assert_codes_close(q, q_ref)
+    np.testing.assert_allclose(s, s_ref, rtol=1e-5)
+
+
+def test_norm_quant_without_transform_degenerate_rows_and_eps():
+    K = 4096
+    x = np.zeros((5, K), dtype=np.float32)
+    x[1, 5] = 3.0
+    x[2] = -1.0
+    x[3, ::2] = 1e-30
+    x[4] = 60000.0 * np.sign(np.sin(np.arange(K)))
+    bits = inputs.f32_to_bf16_bits(x)
+    for quant in QUANT_NAME:
+        abits, mode = QUANT_NAME[quant]
+        for eps_norm, eps_q in ((1e-6, 0.0), (1e-2, 1e-3)):
+            q_ref, s_ref = oracle.norm_fht_quant(bits, None, 1, abits, mode, eps_norm=eps_norm, eps_q=eps_q)
+            q, s = gpu_codes(bits, None, 1, quant, hbl.HBL_CODES_I8, eps_norm=eps_norm, eps_q=eps_q)
+            assert_codes_close(q, q_ref)
+            assert np.all(q[0] == 0) and s[0] == 0.0
+            np.testing.assert_allclose(s[1:], s_ref[1:], rtol=1e-5)
+
+
 @pytest.mark.parametrize("K,fmt", [(2048, hbl.HBL_CODES_I8), (16384, hbl.HBL_CODES_I8),
                                    (16384, hbl.HBL_CODES_PACKED)])
 def test_norm_fht_quant_degenerate_rows(K, fmt):
@@ -157,6 +202,25 @@ def test_pack_weights_matches_oracle(K, N):
     np.testing.assert_array_equal(t2, t8)
     near_half = np.abs(np.abs(W.astype(np.float64) / alpha_ref) - 0.5) < 1e-6
     assert np.all((t8 == t_ref) | near_half)
+    np.testing.assert_array_equal(colsum, t8.astype(np.int64).sum(axis=0))
+
+
+@pytest.mark.parametrize("K,N,had_block", [(256, 256, 0), (2048, 520, 0), (16384, 64, 0), (11008, 64, 256),
+                                           (12288, 40, 4096), (4096, 136, 1), (8192, 2560, 0)])
+def test_pack_weights_rotated_matches_oracle(K, N, had_block):
+    W = np.random.default_rng(K + N + had_block).standard_normal((K, N)).astype(np.float32) * 0.02
+    Wr_ref = oracle.rotate_weights(W, had_block)
+    t_ref, alpha_ref = oracle.absmean_ternarize(Wr_ref)
+    packed, alpha = hbl.hbl_pack_weights_rotated(torch.from_numpy(W).cuda(), had_block)
+    torch.cuda.synchronize()
+    assert alpha == pytest.approx(alpha_ref, rel=1e-6)
+    t2, t8, colsum = decode_blob(packed.cpu().numpy(), K, N)
+    np.testing.assert_array_equal(t2, t8)
+    # the rotation runs in fp32 (relative error ~1e-6 of the column scale): a weight within that
+    # of a rounding boundary may land on either side
+    near_half = np.abs(np.abs(Wr_ref / alpha_ref) - 0.5) < 2e-5
+    assert np.all((t8 == t_ref) | near_half)
+    assert np.count_nonzero(t8 != t_ref) <= max(1, int(1e-4 * t8.size))
     np.testing.assert_array_equal(colsum, t8.astype(np.int64).sum(axis=0))
 
 
@@ -309,6 +373,60 @@ def check_forward(spec, rows=None, out_dtype=hbl.HBL_OUT_F32):
 def test_forward_small(name, M):
     spec = inputs.WORKLOADS[name] if M is None else inputs.WORKLOADS[name].with_m(M)
     check_forward(spec)
+
+
+@pytest.mark.parametrize("M,quant", [(1, hbl.HBL_Q_A4_ABSMEAN), (3, hbl.HBL_Q_A8_ABSMAX), (64, hbl.HBL_Q_A4_ABSMEAN),
+                                     (300, hbl.HBL_Q_A8_ABSMAX), (1024, hbl.HBL_Q_A4_ABSMEAN)])
+def test_plain_bitlinear_forward_qkv_shape(M, quant):
+    # a QKV-like projection 4096 -> 12288 with no rotation (had_block = 1), all rows
+    spec = spec_like("wo_7b_a4", M=M, N=12288, had_block=1, abits=QUANT_NAME[quant][0], seed=11)
+    x = inputs.activations(spec)
+    W = inputs.weights(spec)
+    abits, mode = QUANT_NAME[quant]
+    packed, alpha = hbl.hbl_pack_weights(torch.from_numpy(W).cuda())
+    X = to_dev_bf16(x)
+    Y = hbl.hbl_forward(X, packed, alpha, spec.N, None, 1, quant, out_dtype=hbl.HBL_OUT_F32)
+    codes, s_x = hbl.hbl_norm_fht_quant(X, None, 1, quant, fmt=hbl.HBL_CODES_I8)
+    torch.cuda.synchronize()
+    q_gpu = codes.cpu().numpy().view(np.int8)
+    ref = oracle.h_bitlinear_forward(x, W, None, 1, abits, mode)
+    assert_codes_close(q_gpu, ref["q"])
+    y = Y.cpu().numpy()
+    y_own = oracle.dequant(oracle.ternary_matmul(q_gpu, ref["t"]), ref["s"], ref["alpha"])
+    assert np.all(row_rel_err(y, y_own) <= 1e-5)
+    dq = np.abs(q_gpu.astype(np.float64) - ref["q"])
+    flip_part = (dq @ np.linalg.norm(ref["t"].astype(np.float64), axis=1)) * ref["s"] * ref["alpha"]
+    err = np.linalg.norm(y - ref["y"], axis=1)
+    assert np.all(err <= 1e-3 * np.linalg.norm(ref["y"], axis=1) + flip_part + 1e-30)
+
+
+@pytest.mark.parametrize("name,M", [("wdown_3b_a4", 300), ("wdown_nonpow2_a4", 20), ("wo_7b_a4", 2)])
+def test_forward_with_rotated_weights(name, M):
+    # the weights-and-activations variant: weights rotated by the packer, activations by the layer
+    spec = inputs.WORKLOADS[name].with_m(M)
+    x = inputs.activations(spec)
+    W = inputs.weights(spec)
+    packed, alpha = hbl.hbl_pack_weights_rotated(torch.from_numpy(W).cuda(), spec.had_block)
+    X = to_dev_bf16(x)
+    Y = hbl.hbl_forward(X, packed, alpha, spec.N, None, spec.had_block, hbl.HBL_Q_A4_ABSMEAN)
+    codes, _ = hbl.hbl_norm_fht_quant(X, None, spec.had_block, hbl.HBL_Q_A4_ABSMEAN, fmt=hbl.HBL_CODES_I8)
+    torch.cuda.synchronize()
+    ref = oracle.h_bitlinear_forward(x, W, None, spec.had_block, 4, "absmean", rotate_w=True)
+    assert alpha == pytest.approx(ref["alpha"], rel=1e-6)
+    t2, t8, _ = decode_blob(packed.cpu().numpy(), spec.K, spec.N)
+    q_gpu = codes.cpu().numpy().view(np.int8)
+    assert_codes_close(q_gpu, ref["q"])
+    y = Y.cpu().numpy()
+    # the product of the GPU's own codes with its own weight codes, through the oracle
+    y_own = oracle.dequant(oracle.ternary_matmul(q_gpu, t8), ref["s"], ref["alpha"])
+    assert np.all(row_rel_err(y, y_own) <= 1e-5)
+    # against the oracle end to end: flipped activation codes and weight codes accounted exactly
+    dq = np.abs(q_gpu.astype(np.float64) - ref["q"])
+    dt = np.abs(t8.astype(np.float64) - ref["t"])
+    flip = (dq @ np.linalg.norm(ref["t"].astype(np.float64), axis=1)
+            + np.abs(q_gpu.astype(np.float64)) @ dt.sum(axis=1)) * ref["s"] * ref["alpha"]
+    err = np.linalg.norm(y - ref["y"], axis=1)
+    assert np.all(err <= 1e-3 * np.linalg.norm(ref["y"], axis=1) + flip + 1e-30)
 
 
 FULL = [("single_a8_16x256", None), ("wo_1p3b_a4", None), ("wdown_3b_a4", None), ("wo_7b_a4", 8192),

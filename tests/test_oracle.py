@@ -272,6 +272,46 @@ def test_ternarize_eps_w_closed_form():
     assert not t.any() and alpha == 0.0
 
 
+def test_rotate_weights_undoes_a_rotation():
+    # W = (H / sqrt n) T c along K: rotating it again gives T c (the orthonormal Sylvester matrix
+    # is its own inverse), whose absmean ternarisation is T with alpha = c * mean|T|. A missing
+    # rotation, a transform along N instead of K, or a missing 1/sqrt(n) breaks one of these.
+    K, N, c = 256, 40, 0.013
+    T = RNG.integers(-1, 2, size=(K, N)).astype(np.int8)
+    H = scipy.linalg.hadamard(K) / math.sqrt(K)
+    W = H @ (T.astype(np.float64) * c)
+    Wr = oracle.rotate_weights(W)
+    np.testing.assert_allclose(Wr, T * c, atol=1e-14)
+    t, alpha = oracle.absmean_ternarize(Wr)
+    np.testing.assert_array_equal(t, T)
+    assert alpha == pytest.approx(c * np.abs(T).mean(), rel=1e-12)
+    # block-diagonal: each 256-slice of the K column is rotated on its own
+    W2 = np.kron(np.eye(3), H) @ (np.tile(T, (3, 1)).astype(np.float64) * c)
+    np.testing.assert_allclose(oracle.rotate_weights(W2, 256), np.tile(T, (3, 1)) * c, atol=1e-14)
+
+
+def test_rotate_weights_columns_closed_form():
+    # a unit column e_j becomes column j of the orthonormal Walsh matrix: (-1)^popcount(i & j) / sqrt(n)
+    n, j = 1024, 613
+    W = np.zeros((n, 3))
+    W[j, 1] = 1.0
+    got = oracle.rotate_weights(W)
+    i = np.arange(n)
+    want = np.array([(-1.0) ** bin(int(ii) & j).count("1") for ii in i]) / math.sqrt(n)
+    np.testing.assert_array_equal(got[:, 1], want)
+    assert not got[:, 0].any() and not got[:, 2].any()
+
+
+def test_rotated_layer_keeps_the_full_precision_product():
+    # (H x)^T (H W) = x^T W: rotating both sides leaves the full-precision layer unchanged
+    x = RNG.standard_normal((5, 512))
+    W = RNG.standard_normal((512, 7))
+    xr = oracle.hadamard_transform(x)
+    np.testing.assert_allclose(xr @ oracle.rotate_weights(W), x @ W, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(oracle.hadamard_transform(x, 256) @ oracle.rotate_weights(W, 256), x @ W,
+                               rtol=1e-10, atol=1e-10)
+
+
 # ---------------------------------------------------------------- product
 
 def test_ternary_matmul_brute_force_and_blas():
@@ -401,3 +441,83 @@ def test_planted_norm_and_rounding_mistakes_are_caught(monkeypatch):
     monkeypatch.setattr(oracle.hbl_oracle, "_round_clip", half_away)
     with pytest.raises(AssertionError):
         test_quantiser_ties_go_to_even()
+
+
+
+# ---------------------------------------------------------------- QKV states after RoPE
+
+def test_rope_identity_norm_and_inverse():
+    x = RNG.standard_normal((6, 3, 128))
+    pos = np.array([0, 1, 7, 100, 4095, 8191])
+    y = oracle.rope(x, pos)
+    np.testing.assert_array_equal(y[0], x[0])  # position 0: angle 0
+    # every (f, f + D/2) pair keeps its length
+    n_x = x[..., :64] ** 2 + x[..., 64:] ** 2
+    n_y = y[..., :64] ** 2 + y[..., 64:] ** 2
+    np.testing.assert_allclose(n_y, n_x, rtol=1e-12)
+    # rotating by -pos undoes it
+    np.testing.assert_allclose(oracle.rope(y, -pos), x, atol=1e-12)
+
+
+def test_rope_one_hot_closed_form():
+    D, f, p, theta = 64, 5, 37, 10000.0
+    x = np.zeros((1, 1, D))
+    x[0, 0, f] = 1.0
+    y = oracle.rope(x, np.array([p]), theta)[0, 0]
+    a = p * theta ** (-2.0 * f / D)
+    want = np.zeros(D)
+    want[f], want[f + D // 2] = math.cos(a), math.sin(a)
+    np.testing.assert_allclose(y, want, atol=1e-15)
+    x = np.zeros((1, 1, D))
+    x[0, 0, f + D // 2] = 1.0  # the second feature of the pair turns the other way
+    y = oracle.rope(x, np.array([p]), theta)[0, 0]
+    want = np.zeros(D)
+    want[f], want[f + D // 2] = -math.sin(a), math.cos(a)
+    np.testing.assert_allclose(y, want, atol=1e-15)
+
+
+def test_rope_depends_on_relative_position():
+    # <rope(q, p), rope(k, p')> depends on p - p' only (brute force over position pairs)
+    q = RNG.standard_normal((1, 1, 128))
+    k = RNG.standard_normal((1, 1, 128))
+    for p, pp in ((10, 3), (1000, 993), (5, -2)):
+        a = np.sum(oracle.rope(q, np.array([p])) * oracle.rope(k, np.array([pp])))
+        b = np.sum(oracle.rope(q, np.array([p - pp])) * k)
+        assert a == pytest.approx(b, rel=1e-10)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_unsigned_quantiser_properties(bits):
+    L = (1 << bits) - 1
+    x = RNG.standard_normal((40, 4, 128))
+    u, g = oracle.quantize_unsigned_absmax(x, bits)
+    assert u.dtype == np.uint8 and u.min() >= 0 and u.max() <= L
+    np.testing.assert_array_equal(g, np.abs(x).max(axis=-1))
+    # the element of largest magnitude maps to an end of the range
+    am = np.abs(x).argmax(axis=-1)
+    ext = np.take_along_axis(u, am[..., None], axis=-1)[..., 0]
+    sgn = np.sign(np.take_along_axis(x, am[..., None], axis=-1)[..., 0])
+    np.testing.assert_array_equal(ext, np.where(sgn > 0, L, 0))
+    # dequantised values lie within half a step (gamma / L) of x, and the code is the nearest
+    # level, found here by searching all 2^b levels
+    xd = oracle.dequantize_unsigned(u, g, bits)
+    assert np.all(np.abs(xd - x) <= g[..., None] / L * (1 + 1e-12))
+    levels = (2.0 * np.arange(L + 1) - L) / L
+    xs, gs, us = x[:2].reshape(-1, 128), g[:2].reshape(-1), u[:2].reshape(-1, 128)
+    for h in range(xs.shape[0]):
+        for d in range(128):
+            best = int(np.argmin(np.abs(levels * gs[h] - xs[h, d])))
+            assert us[h, d] == best
+
+
+def test_unsigned_quantiser_closed_form():
+    # b = 3: [-gamma, gamma] onto 0..7, step 2 gamma / 7. x = [-1, 1, 0, 0.5, -0.25] (gamma = 1):
+    # 3.5 (x + 1) = [0, 7, 3.5, 5.25, 2.625] -> [0, 7, 4 (tie to even), 5, 3]
+    u, g = oracle.quantize_unsigned_absmax(np.array([[-1.0, 1.0, 0.0, 0.5, -0.25]]), 3)
+    np.testing.assert_array_equal(u[0], [0, 7, 4, 5, 3])
+    assert g[0] == 1.0
+    np.testing.assert_allclose(oracle.dequantize_unsigned(u, g, 3)[0], [-1, 1, 1 / 7, 3 / 7, -1 / 7], rtol=1e-15)
+    # a zero head takes the middle code and dequantises to 0
+    u, g = oracle.quantize_unsigned_absmax(np.zeros((1, 8)), 3)
+    assert np.all(u == 4) and g[0] == 0.0
+    assert not oracle.dequantize_unsigned(u, g, 3).any()
