@@ -153,19 +153,19 @@ constexpr int eb_for(int L) {
   return L == 8 ? 4 : L == 9 ? 5 : L == 10 ? 5 : L == 11 ? 6 : L == 12 ? 6 : 7;
 }
 
-// Transforms of 2^L features (one block, no gain) with the H_128 factor on the tensor cores; the
-// grid walks groups of 2^(14-L) rows, two CTAs per SM.
-template <int QM, int L>
+// The tensor-core activation kernel: groups of R rows in one 16384-element buffer, transform
+// blocks of 2^LB features; the grid walks the groups, two CTAs per SM.
+template <int QM, int R, int LB>
 hbl_status launch_nfq_tc(const NfqArgs& a, cudaStream_t s) {
   static SmemLimit lim;
-  auto* k = norm_fht_quant_tc_kernel<QM, L>;
+  auto* k = norm_fht_quant_tc_kernel<QM, R, LB>;
   cudaError_t e = allow_smem(k, kNtSmem, lim);
   if (e != cudaSuccess) return cuda_fail(e);
   cudaLaunchConfig_t cfg = {};
   int dev = 0;
   cudaGetDevice(&dev);
   const int resident = kNtCtasPerSm * device_sms(dev);
-  const int groups = (a.M + (kNtN >> L) - 1) / (kNtN >> L);  // 2^(14-L) rows per group
+  const int groups = (a.M + R - 1) / R;
   cfg.gridDim = dim3(groups < resident ? groups : resident, 1, 1);
   cfg.blockDim = dim3(kNtThreads, 1, 1);
   cfg.dynamicSmemBytes = kNtSmem;
@@ -281,19 +281,24 @@ hbl_status run_nfq(const void* X, const float* gain, int M, int K, int had_block
   a.groups = (M + rows - 1) / rows;
   a.pf_dist = 0;
 
-  // One block of 2^12 .. 2^14 features, no gain: the tensor-core kernel. (It also serves 2^11
-  // correctly; an earlier version of its per-row epilogue measured slower there than the CUDA-core
-  // kernel, 12.5 against 7.1 us on 2048 x 2048, so 2^11 stays on CUDA cores until measured again.)
-  if (L >= 12 && L <= 14 && nb == 1 && gain == nullptr) {
-    auto tc = [&](auto lc) -> hbl_status {
-      constexpr int LL = decltype(lc)::value;
-      if (quant == 0) return launch_nfq_tc<0, LL>(a, stream);
-      if (quant == 1) return launch_nfq_tc<1, LL>(a, stream);
-      return launch_nfq_tc<2, LL>(a, stream);
+  // The tensor-core kernel (no gain): one block of 2^12 .. 2^14 features in groups of 16384 / K
+  // rows, or blocks of 256 features in rows of at most 16384 features that are not a power of two,
+  // one row per group. (It also serves one block of 2^11 correctly; an earlier version of its
+  // per-row epilogue measured slower there than the CUDA-core kernel, 12.5 against 7.1 us on
+  // 2048 x 2048, so 2^11 stays on CUDA cores until measured again.)
+  if (gain == nullptr) {
+    auto tc = [&](auto rc, auto lc) -> hbl_status {
+      constexpr int RR = decltype(rc)::value, LL = decltype(lc)::value;
+      if (quant == 0) return launch_nfq_tc<0, RR, LL>(a, stream);
+      if (quant == 1) return launch_nfq_tc<1, RR, LL>(a, stream);
+      return launch_nfq_tc<2, RR, LL>(a, stream);
     };
-    if (L == 12) return tc(std::integral_constant<int, 12>{});
-    if (L == 13) return tc(std::integral_constant<int, 13>{});
-    return tc(std::integral_constant<int, 14>{});
+    using std::integral_constant;
+    if (nb == 1 && L == 12) return tc(integral_constant<int, 4>{}, integral_constant<int, 12>{});
+    if (nb == 1 && L == 13) return tc(integral_constant<int, 2>{}, integral_constant<int, 13>{});
+    if (nb == 1 && L == 14) return tc(integral_constant<int, 1>{}, integral_constant<int, 14>{});
+    if (nb > 1 && L == 8 && K <= 16384 && !is_pow2(K))
+      return tc(integral_constant<int, 1>{}, integral_constant<int, 8>{});
   }
   // K <= 32768 bounds nb, so these R always suffice: L=8 nb<=128 (R<=4), L=9..12 R<=2, L>=13 R=1
   switch (L) {

@@ -1,35 +1,41 @@
-// Fused RMSNorm -> fast Walsh-Hadamard transform -> per-token quantisation for 16384-wide rows,
-// with the first Kronecker factor of the transform on the tensor cores.
+// Fused RMSNorm -> fast Walsh-Hadamard transform -> per-token quantisation with the first
+// Kronecker factor of the transform on the tensor cores.
 //
 // Method: BitNet v2 walkthrough article (m.jxzklqfsx.com), section "H-BitLinear模塊": an online
 // Hadamard transform of the normalised activations before per-token quantisation; the page
 // defines the transform as a matrix product computed with the fast Hadamard transform.
 //
-// H_16384 = H_128 (x) H_128 in Sylvester order: H[k][k'] = (-1)^popcount(k & k') factors over
-// any split of the 14 index bits. Split k into the 7 bits a = (k bits 13..10, 5..3) and the 7
-// bits n = (k bits 9..6, 2..0):
-//   y[a, n] = sum_{a'} H_128[a][a'] * sum_{n'} H_128[n][n'] * x[a', n'],
-// and the two factors commute. On CUDA cores the 14 butterfly stages cost 14 fp32 adds per
-// element and bound the kernel by the FP32 pipe and issue, not by HBM; here the factor over a is
-// one exact tensor-core product per row,
-//   D[a][n] = sum_{a'} H_128[a][a'] * x[a', n]    (tcgen05.mma kind::f16, bf16 x bf16 -> fp32),
-// exact up to fp32 rounding since x is bf16 and H is +-1, and the factor over n is 7 butterfly
-// stages on CUDA cores. The MMA's B operand is the bf16 row itself, as the TMA copy lands it,
-// read MN-major: the 128 contiguous bytes of features 64j .. 64j + 63 are one 8 x 16-byte core
-// matrix whose 16-byte rows hold 8 consecutive n (k bits 2..0) and step through a' (k bits
-// 5..3); core matrices lie 128 bytes apart along N (k bits 9..6) and 2048 bytes apart along K
-// (k bit 10). TMEM lane a of the accumulator then holds, in its 128 columns, exactly the values
-// one thread needs for the remaining stages, and after them 16 runs of 8 consecutive outputs:
-// the thread forms its codes and stores them to global memory directly, with no regrouping
-// through shared memory.
+// A group of R rows (R K <= 16384) lands in one 16384-element bf16 buffer; element index
+// e = 1024 nh + 8 a + nl splits into a = e bits 9..3 (7 bits) and the column c = (nh, nl). The
+// Sylvester matrix H[k][k'] = (-1)^popcount(k & k') factors over any split of the index bits, so
+// the transform of each block of HB = 2^LB features is
+//   D[a][c] = sum_{a'} A[a][a'] * buf[a', c]    (tcgen05.mma kind::f16, bf16 x bf16 -> fp32),
+// with A = I (x) H_P (P = min(HB / 8, 128): the index bits 9..3 that lie inside a block; the
+// others are block-index bits and get the identity), followed by butterfly stages on CUDA cores
+// over the remaining in-block bits: nl (k bits 2..0) and, for blocks of 2048 .. 16384, k bits
+// 10 .. LB - 1. The product is exact up to fp32 rounding since buf is bf16 and A is 0/+-1. For one
+// block of 4096 .. 16384 features this is H_128 on the tensor cores; for K = 43 x 256 (blocks of
+// 256, one row per group) it is I_4 (x) H_32 and three stages. Columns past the end of a row hold
+// zeros (the buffer's tail is cleared once per CTA) and are neither counted nor stored.
+// On CUDA cores alone the 14 butterfly stages of a 16384-point transform cost 14 fp32 adds per
+// element and bound the kernel by the FP32 pipe and issue, not by HBM.
 //
-//   warps 0-3  consumers, thread = TMEM lane a: tcgen05.ld of the 128 columns, 7 butterfly
-//              stages, row statistics (one named barrier), quantisation, 16 stores of 8 codes
-//   warp 4     TMEM allocation; one thread copies rows in (one 32 KB bulk copy each) and issues
-//              the 8 MMAs (K = 16 each) of a row into one of two TMEM accumulators
-// Persistent CTAs (two per SM) walk the rows. (With the consumers' arithmetic taken out the copies
-// and MMAs alone run at 5.2 TB/s: the consumers are the limit.) Every mbarrier wait is bounded
-// (1 s); the consumers vote on the outcome of their waits so that they leave their loop together.
+// The MMA's B operand is the bf16 buffer itself, as the bulk copy lands it, read MN-major: the 128
+// contiguous bytes of features 64j .. 64j + 63 are one 8 x 16-byte core matrix whose 16-byte rows
+// hold 8 consecutive nl and step through a' (e bits 5..3); core matrices lie 128 bytes apart along
+// N (e bits 9..6) and 2048 bytes apart along K (e bit 10). TMEM lane a of the accumulator then
+// holds, in its 128 columns, exactly the values one thread needs for the remaining stages, and
+// after them runs of 8 consecutive outputs: the thread forms its codes and stores them to global
+// memory directly, with no regrouping through shared memory.
+//
+//   warps 0-3  consumers, thread = TMEM lane a: tcgen05.ld of the 128 columns, the remaining
+//              butterfly stages, row statistics (one named barrier), quantisation, stores of 8 codes
+//   warp 4     TMEM allocation; one thread copies groups in (one bulk copy each) and issues the 8
+//              MMAs (K = 16 each) of a group into one of two TMEM accumulators
+// Persistent CTAs (two per SM) walk the groups. (With the consumers' arithmetic taken out the
+// copies and MMAs alone run at 5.2 TB/s: the consumers are the limit.) Every mbarrier wait is
+// bounded (1 s); the consumers vote on the outcome of their waits so that they leave their loop
+// together.
 #pragma once
 
 #include "common.cuh"
@@ -38,8 +44,8 @@
 
 namespace hbl {
 
-constexpr int kNtN = 16384;                       // features in one group (16384 / K rows)
-constexpr int kNtRowBytes = kNtN * 2;             // the group's bf16 landing buffer
+constexpr int kNtN = 16384;                       // transform size (the whole row)
+constexpr int kNtRowBytes = kNtN * 2;             // one bf16 row
 constexpr int kNtThreads = 160;                   // 4 consumer warps + 1 copy / MMA warp
 constexpr int kNtTmemCols = 256;                  // two 128-column fp32 accumulators
 constexpr int kNtSmem = 32768 + kNtRowBytes + 1024;  // H, rows, alignment slack
@@ -147,9 +153,11 @@ __device__ __forceinline__ uint32_t codes4(float2 va, float2 vb, float2 mult2) {
 // feature) contiguous bytes.
 template <int CM, int RUNS>
 __device__ __forceinline__ void quant_store(const float2* v, float2 mult2, uint8_t* row_codes, bool packed4,
-                                            int a) {
+                                            int a, int K) {
 #pragma unroll
   for (int u = 0; u < RUNS; ++u) {
+    if (1024 * u >= K) break;            // past the row: the same in every lane
+    if (1024 * u + 8 * a >= K) continue;  // the row ends inside this 1024-feature chunk
     const uint32_t w0 = codes4<CM>(v[4 * u], v[4 * u + 1], mult2);
     const uint32_t w1 = codes4<CM>(v[4 * u + 2], v[4 * u + 3], mult2);
     if (!packed4) {
@@ -163,14 +171,20 @@ __device__ __forceinline__ void quant_store(const float2* v, float2 mult2, uint8
   }
 }
 
-// QM: 0 = a8 absmax, 1 = a4 absmean, 2 = a4 absmax. L: log2 K, 11..14; a group of 2^(14-L) rows.
-template <int QM, int L>
+// QM: 0 = a8 absmax, 1 = a4 absmean, 2 = a4 absmax. R: rows per group (R K <= 16384; a row
+// shorter than 16384 features that is not a power of two is a group of its own, the rest of the
+// buffer zero). LB: log2 of the transform block (K = nb 2^LB).
+template <int QM, int R, int LB>
 __global__ void __launch_bounds__(kNtThreads, kNtCtasPerSm) norm_fht_quant_tc_kernel(const NfqArgs a) {
-  static_assert(L >= 11 && L <= 14, "the group must fill 16384 elements with at most 8 rows");
-  constexpr int K = 1 << L;
-  constexpr int R = kNtN / K;   // rows per group
-  constexpr int NB = K / 128;   // accumulator columns (values of n) per row
+  static_assert(R == 1 || R == 2 || R == 4 || R == 8, "rows per group");
+  static_assert(LB >= 8 && LB <= 14, "transform block");
+  constexpr int HB = 1 << LB;
+  constexpr int LP = LB - 3 < 7 ? LB - 3 : 7;  // the tensor-core factor I (x) H_P over k bits 9..3
+  constexpr int P = 1 << LP;
+  constexpr int NST = 3 + (LB > 10 ? LB - 10 : 0);  // butterfly stages left: k bits 2..0, 10..LB-1
+  constexpr int NB = 128 / R;   // accumulator columns per row
   constexpr int RUNS = NB / 8;  // runs of 8 consecutive features per row and thread
+  const int K = a.K;
   extern __shared__ __align__(1024) uint8_t smem_nt[];
   __shared__ __align__(8) uint64_t land_full, land_empty, acc_full[2], acc_empty[2], drain_bar;
   __shared__ uint32_t tmem_slot;
@@ -211,16 +225,27 @@ __global__ void __launch_bounds__(kNtThreads, kNtCtasPerSm) norm_fht_quant_tc_ke
     if (ng > 0) copy_group((int)blockIdx.x);
   }
 
-  // ---- H_128 in the A-operand layout: element (a, a') = (-1)^popcount(a & a') as bf16, a' in
-  // two halves of 64; within a half, 16-byte chunk c of row a sits at chunk c ^ (a & 7)
+  // ---- I (x) H_P in the A-operand layout: element (a, a') = (-1)^popcount(a & a') as bf16 where
+  // a and a' lie in the same block of P, else 0; a' in two halves of 64; within a half, 16-byte
+  // chunk c of row a sits at chunk c ^ (a & 7)
+  auto hval = [](int r, int k) -> uint32_t {
+    if ((r >> LP) != (k >> LP)) return 0u;
+    return (__popc(r & k & (P - 1)) & 1) ? 0xbf80u : 0x3f80u;  // the block bits carry no sign
+  };
   for (int e = tid; e < 128 * 64; e += kNtThreads) {  // two elements per 32-bit store
     const int r = e >> 6, k0 = (e & 63) * 2;
-    const uint32_t v0 = (__popc(r & k0) & 1) ? 0xbf80u : 0x3f80u;
-    const uint32_t v1 = (__popc(r & (k0 + 1)) & 1) ? 0xbf80u : 0x3f80u;
+    const uint32_t v0 = hval(r, k0);
+    const uint32_t v1 = hval(r, k0 + 1);
     const int half = k0 >> 6, kh = k0 & 63;
     *reinterpret_cast<uint32_t*>(hA + half * 16384 + r * 128 + (((kh >> 3) ^ (r & 7)) << 4) + (kh & 7) * 2) =
         v0 | (v1 << 16);
   }
+  // a row shorter than the buffer: the tail stays zero (copies write only the first K features),
+  // so the columns past the row hold exact zeros -- a stale NaN there would reach the valid
+  // outputs of its column through the zeros of I (x) H_P
+  if (R * K < kNtN)
+    for (int e = R * K * 2 + tid * 16; e < kNtRowBytes; e += kNtThreads * 16)
+      *reinterpret_cast<uint4*>(land + e) = make_uint4(0u, 0u, 0u, 0u);
   fence_proxy_async_shared();  // generic-proxy writes -> visible to the tensor core
   if (warp == 4) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -319,7 +344,7 @@ __global__ void __launch_bounds__(kNtThreads, kNtCtasPerSm) norm_fht_quant_tc_ke
         }
       }
 
-      fwht_regs2<128, L - 7>(v);  // the factor over n, within each row
+      fwht_regs2<128, NST>(v);  // the factor over n within each block
 
       if constexpr (kAbsmax) {
         float acc[R * PER];
@@ -384,8 +409,8 @@ __global__ void __launch_bounds__(kNtThreads, kNtCtasPerSm) norm_fht_quant_tc_ke
         const float ssr = (rs_[0] + rs_[1]) + (rs_[2] + rs_[3]);
         const float str = kAbsmax ? fmaxf(fmaxf(rt_[0], rt_[1]), fmaxf(rt_[2], rt_[3]))
                                   : (rt_[0] + rt_[1]) + (rt_[2] + rt_[3]);
-        const float r_rms = sqrtf(ssr / (128.f * (float)K) + a.eps_norm);
-        const float rs = r_rms * sqrtf((float)K);
+        const float r_rms = sqrtf(ssr / ((float)P * (float)K) + a.eps_norm);  // sum D^2 = P sum x^2
+        const float rs = r_rms * sqrtf((float)HB);
         const float sy = kAbsmax ? str : str / (float)K;
         if (a.eps_q == 0.f) {
           mult_l = sy > 0.f ? kQ / sy : 0.f;
@@ -396,9 +421,10 @@ __global__ void __launch_bounds__(kNtThreads, kNtCtasPerSm) norm_fht_quant_tc_ke
           sx_l = stat / kQ;
         }
         // the absmean clamp may run on 16-bit lanes when every rounded product fits an int16:
-        // |y mult| <= mult ||y||_2 and ||y||_2^2 = NB ssr (the n stages scale the sum of squares by
-        // NB), so mult sqrt(NB ssr) < 30000 guarantees it with room for fp32 rounding
-        lanes16_l = mult_l * sqrtf((float)NB * ssr) < 30000.f ? 1 : 0;
+        // |y mult| <= mult ||y||_2 and ||y||_2^2 = (HB / P) ssr (the remaining stages scale the sum
+        // of squares by HB / P), so mult sqrt(HB / P ssr) < 30000 guarantees it with room for fp32
+        // rounding
+        lanes16_l = mult_l * sqrtf((float)(HB / P) * ssr) < 30000.f ? 1 : 0;
       }
       if (warp == 0 && lane < R && g * R + lane < a.M) a.s_x[g * R + lane] = sx_l;
 
@@ -412,11 +438,11 @@ __global__ void __launch_bounds__(kNtThreads, kNtCtasPerSm) norm_fht_quant_tc_ke
         const float2* vr = v + r * (NB / 2);
         uint8_t* row_codes = a.codes + (size_t)row * (packed4 ? K / 2 : K);
         if constexpr (kAbsmax) {
-          quant_store<0, RUNS>(vr, mult2, row_codes, packed4, arow);
+          quant_store<0, RUNS>(vr, mult2, row_codes, packed4, arow, K);
         } else if (lanes16) {
-          quant_store<1, RUNS>(vr, mult2, row_codes, packed4, arow);
+          quant_store<1, RUNS>(vr, mult2, row_codes, packed4, arow, K);
         } else {
-          quant_store<2, RUNS>(vr, mult2, row_codes, packed4, arow);
+          quant_store<2, RUNS>(vr, mult2, row_codes, packed4, arow, K);
         }
       }
     }

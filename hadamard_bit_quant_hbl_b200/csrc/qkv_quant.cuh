@@ -5,8 +5,8 @@
 // QKV states are quantised after RoPE; each head goes directly to unsigned integers through the
 // absmax function, with no calibration data. The formulas were not preserved, so this follows the
 // plainest reading: per token and head, gamma = max|x| over the head's D features, and
-// [-gamma, gamma] maps linearly onto [0, 2^b - 1]:
-//     u = RoundClip((2^b - 1)/2 * (x/gamma + 1), 0, 2^b - 1),   x~ = (2u - (2^b - 1)) gamma/(2^b - 1).
+// [-gamma, gamma] maps linearly onto [0, 2^b - 1] (L = 2^b - 1):
+//     u = RoundClip(L (x + gamma) / (2 gamma), 0, L),   x~ = (2u - L) gamma / L.
 // RoPE is the LLaMA form of the model's LLaMA-like parts ("BitNet v2：原生4位激活"): feature f of a
 // head pairs with f + D/2 and both turn by the angle pos * theta^(-2f/D).
 //
@@ -116,11 +116,15 @@ __global__ void __launch_bounds__(256) qkv_quant_kernel(QkvArgs a) {
     for (int e = 0; e < E; ++e) g = fmaxf(g, fabsf(v[e]));
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, o));
-    const float mult = g > 0.f ? 0.5f * kL / g : 0.f;
+    // u = rint(L (x + gamma) / (2 gamma)): the numerator by one fused multiply-add (exact for bf16
+    // inputs, whose products with L need 16 bits), then a correctly rounded division, so that a
+    // value exactly on a .5 boundary stays on it and goes to the even code
+    const float lg = kL * g, den = 2.f * g;
     unsigned long long bits = 0;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-      const float q = fminf(fmaxf(rintf(fmaf(v[e], mult, 0.5f * kL)), 0.f), kL);
+      const float t = g > 0.f ? __fdiv_rn(fmaf(kL, v[e], lg), den) : 0.5f * kL;
+      const float q = fminf(fmaxf(rintf(t), 0.f), kL);
       bits |= (unsigned long long)(uint32_t)q << (((lane % LPG) * E + e) * BITS);
     }
 #pragma unroll

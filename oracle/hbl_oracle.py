@@ -44,10 +44,9 @@ Readings taken where the pages are silent or the formulas were dropped
      pos * theta^(-2f/D); theta is a parameter (10000 by default).
   R9 QKV quantisation after RoPE to unsigned b-bit integers with an absmax scale, per
      token and head: gamma = max|x| over the head's D values, the interval
-     [-gamma, gamma] mapped linearly onto [0, 2^b - 1]:
-       u = RoundClip((2^b - 1)/2 * (x/gamma + 1), 0, 2^b - 1),
-       x~ = (2u - (2^b - 1)) * gamma / (2^b - 1);
-     a head whose gamma is 0 takes x/gamma = 0.
+     [-gamma, gamma] mapped linearly onto [0, L], L = 2^b - 1:
+       u = RoundClip(L (x + gamma) / (2 gamma), 0, L),   x~ = (2u - L) gamma / L;
+     a head whose gamma is 0 takes u = RoundClip(L / 2).
 
 Parity status: every function below names the tests that pin it against
 something other than itself (closed forms, a dense Sylvester matrix from
@@ -320,10 +319,14 @@ def quantize_unsigned_absmax(x: np.ndarray, bits: int) -> tuple[np.ndarray, np.n
     """
     x = np.asarray(x, dtype=np.float64)
     L = (1 << bits) - 1
-    g = np.abs(x).max(axis=-1)
-    r = np.where(g[..., None] > 0, x / np.where(g > 0, g, 1.0)[..., None], 0.0)
-    u = np.clip(np.rint(L / 2.0 * (r + 1.0)), 0, L).astype(np.uint8)
-    return u, g
+    g = np.abs(x).max(axis=-1)[..., None]
+    live = g > 0
+    gs = np.where(live, g, 1.0)
+    # L (x + gamma) / (2 gamma) in one division: for bf16 inputs the numerator is exact in float64,
+    # so a value exactly on a .5 boundary is represented exactly and goes to the even code
+    v = np.where(live, (L * x + L * gs) / (2.0 * gs), L / 2.0)
+    u = np.clip(np.rint(v), 0, L).astype(np.uint8)
+    return u, g[..., 0]
 
 
 def dequantize_unsigned(u: np.ndarray, gamma: np.ndarray, bits: int) -> np.ndarray:

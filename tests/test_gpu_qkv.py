@@ -78,12 +78,16 @@ def test_qkv_quant_degenerate_heads_and_theta():
     x[1, 128 + 7] = -2.5           # one spike: gamma = 2.5, every other feature the middle code
     x[2, :128] = 1.0               # a constant head
     x[2, 256:384] = np.linspace(-3, 3, 128)
+    x[0, 384:390] = [1.5625, 0.625, -0.625, 1.25, -1.25, 0.0]  # exact .5 ties at 8 bits (no rotation)
     bits = inputs.f32_to_bf16_bits(x)
     pos = np.array([0, 5, 4000])
     for b in (2, 3, 4, 8):
         u, g = check(bits, H, D, b, pos, theta=500000.0)
-        assert np.all(g[0] == 0.0)
-        assert np.all(u[0] == (1 << (b - 1)))  # zero heads: the code nearest the middle (ties to even)
+        assert np.all(g[0, :3] == 0.0)
+        assert np.all(u[0, :3] == (1 << (b - 1)))  # zero heads: the code nearest the middle (ties to even)
+        u, g = check(bits, H, D, b, None)  # no rotation: the ties of row 0, head 3 are exact
+        if b == 8:
+            np.testing.assert_array_equal(u[0, 3, :6], [255, 178, 76, 230, 26, 128])
 
 
 def test_qkv_quant_full_size_7b_heads():

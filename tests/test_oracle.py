@@ -521,3 +521,7 @@ def test_unsigned_quantiser_closed_form():
     u, g = oracle.quantize_unsigned_absmax(np.zeros((1, 8)), 3)
     assert np.all(u == 4) and g[0] == 0.0
     assert not oracle.dequantize_unsigned(u, g, 3).any()
+    # exact ties at b = 8 go to the even code: with gamma = 1.5625 (all values bf16), 255 (x + gamma)
+    # / (2 gamma) is exactly 178.5, 76.5, 229.5 and 25.5 for x = 0.625, -0.625, 1.25, -1.25
+    u, _ = oracle.quantize_unsigned_absmax(np.array([[1.5625, 0.625, -0.625, 1.25, -1.25, 0.0]]), 8)
+    np.testing.assert_array_equal(u[0], [255, 178, 76, 230, 26, 128])
