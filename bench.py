@@ -471,6 +471,9 @@ def run_ours(args, world, rank, local):
                      "achieved": gemm_ops / (per[2 * i + 1] / 1e3) / 1e12, "unit": "TOP/s",
                      "frac": gemm_ops / (per[2 * i + 1] / 1e3) / 1e12 / int8_peak_tops})
     dom = max(kern, key=lambda k: k["ms"])
+    # algorithmic bytes of the dominant (Wdown) product: a4 codes, 2-bit weights, bf16 output
+    dom_layer = layers[-1]["spec"]
+    dom_bytes = dom_layer.M * dom_layer.K // 2 + dom_layer.K * dom_layer.N // 4 + 2 * dom_layer.M * dom_layer.N
     traffic = None
     rec = NCU_TRAFFIC.get(dom["kernel"])
     if rec and src_hash(rec["src"]) == rec["sha"]:  # null once the kernel source has changed
@@ -495,8 +498,14 @@ def run_ours(args, world, rank, local):
                      "peak": int8_peak_tops if dom["bound"] == "tensor" else hbm,
                      "unit": "TOP/s" if dom["bound"] == "tensor" else "GB/s", "frac": dom["frac"],
                      "traffic": traffic, "kernel": dom["kernel"],
-                     "peak_source": (f"{peak_src} bf16 burst x2 (int8:bf16 nominal ratio)"
-                                     if dom["bound"] == "tensor" else f"{peak_src} HBM copy")},
+                     "peak_source": (f"{peak_src} bf16 burst x2 (int8:bf16 nominal ratio; the timed region is "
+                                     f"short, so the burst figure applies)"
+                                     if dom["bound"] == "tensor" else f"{peak_src} HBM copy"),
+                     "frac_of_sustained_peak": (dom["achieved"] / (2.0 * bf16_sus) if dom["bound"] == "tensor"
+                                                else None),
+                     "algorithmic_bytes": dom_bytes,
+                     "traffic_note": "DRAM bytes above the algorithmic ones: A tiles re-read per 256-column tile "
+                                     "and weights read as int8 (the kernel is bound by the tensor pipe)"},
         "kernels": kern,
         "e2e": ({"value": tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                  "d2h_bytes_per_step": d2h} if e2e_steps else None),
@@ -660,6 +669,67 @@ def run_profile_product(M):
     print(f"product {product_kernel(M)[0]}: M={M} K={spec.K} N={spec.N}, 3 launches", flush=True)
 
 
+def run_profile_activation(name, M):
+    """Runs the fused activation kernel (a4 absmean, int8 codes) three times on one workload with
+    M tokens: a small, self-contained target for an ncu capture; no bench line."""
+    import torch
+
+    import hadamard_bit_quant_hbl_b200 as hbl
+
+    torch.cuda.set_device(0)
+    spec = inputs.WORKLOADS[name].with_m(M)
+    quant = hbl.HBL_Q_A8_ABSMAX if spec.abits == 8 else hbl.HBL_Q_A4_ABSMEAN
+    X = torch.from_numpy(inputs.activations(spec).view(np.int16)).cuda().view(torch.bfloat16)
+    codes = torch.empty((M, spec.K), dtype=torch.uint8, device="cuda")
+    s_x = torch.empty(M, dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        hbl.hbl_norm_fht_quant(X, None, spec.had_block, quant, 1e-6, 0.0, hbl.HBL_CODES_I8, codes, s_x)
+    torch.cuda.synchronize()
+    st = hbl.hbl_device_status()
+    if st != hbl.HBL_OK:
+        raise RuntimeError(hbl.hbl_status_string(st))
+    print(f"activation {nfq_kernel(spec.K, spec.had_block)}: {name} M={M} K={spec.K}, 3 launches", flush=True)
+
+
+def run_profile_forward(M, name="wdown_7b_a4"):
+    """Runs hbl_forward three times on one workload with M tokens (one token of K <= 8192 is the
+    fused decode kernel: one launch per layer); an ncu target, no bench line."""
+    import torch
+
+    import hadamard_bit_quant_hbl_b200 as hbl
+
+    torch.cuda.set_device(0)
+    spec = inputs.WORKLOADS[name].with_m(M)
+    X = torch.from_numpy(inputs.activations(spec).view(np.int16)).cuda().view(torch.bfloat16)
+    packed, alpha = hbl.hbl_pack_weights(torch.from_numpy(inputs.weights(spec)).cuda())
+    for _ in range(3):
+        hbl.hbl_forward(X, packed, alpha, spec.N, None, 0, hbl.HBL_Q_A4_ABSMEAN, out_dtype=hbl.HBL_OUT_BF16)
+    torch.cuda.synchronize()
+    st = hbl.hbl_device_status()
+    if st != hbl.HBL_OK:
+        raise RuntimeError(hbl.hbl_status_string(st))
+    print(f"forward: {name} M={M}, 3 calls", flush=True)
+
+
+def run_profile_qkv(M, H=32, D=128, bits=3):
+    """Runs the post-RoPE QKV quantiser three times on M tokens x H heads x D (positions 0..M-1):
+    an ncu target; no bench line."""
+    import torch
+
+    import hadamard_bit_quant_hbl_b200 as hbl
+
+    torch.cuda.set_device(0)
+    X = torch.from_numpy(inputs.qkv_states(M, H, D).view(np.int16)).cuda().view(torch.bfloat16)
+    pos = torch.arange(M, dtype=torch.int32, device="cuda")
+    for _ in range(3):
+        hbl.hbl_qkv_quant(X, H, D, bits, pos=pos)
+    torch.cuda.synchronize()
+    st = hbl.hbl_device_status()
+    if st != hbl.HBL_OK:
+        raise RuntimeError(hbl.hbl_status_string(st))
+    print(f"qkv_quant: M={M} H={H} D={D} bits={bits}, 3 launches", flush=True)
+
+
 ACTIVATION_CASES = [("wo_7b_a4", 8192), ("wdown_7b_a4", 8192), ("wdown_3b_a4", 4096),
                     ("wdown_nonpow2_a4", 8192), ("wo_1p3b_a4", 2048), ("qkv_7b_plain_a4", 8192)]
 
@@ -732,9 +802,25 @@ def main():
                     help="only run the Wdown product three times with M tokens (an ncu target); no bench line")
     ap.add_argument("--activation-only", action="store_true",
                     help="only time the fused activation kernel alone on each workload width; no bench line")
+    ap.add_argument("--profile-activation", nargs=2, metavar=("WORKLOAD", "M"),
+                    help="only run the activation kernel of one workload three times (an ncu target)")
+    ap.add_argument("--profile-forward", nargs="+", metavar=("M", "WORKLOAD"),
+                    help="only run hbl_forward three times with M tokens on a workload (default the 7B Wdown; "
+                         "an ncu target)")
+    ap.add_argument("--profile-qkv", type=int, default=0, metavar="M",
+                    help="only run the QKV quantiser three times on M tokens x 32 heads x 128 (an ncu target)")
     args = ap.parse_args()
     if args.activation_only:
         run_activation_only()
+        return
+    if args.profile_activation:
+        run_profile_activation(args.profile_activation[0], int(args.profile_activation[1]))
+        return
+    if args.profile_qkv:
+        run_profile_qkv(args.profile_qkv)
+        return
+    if args.profile_forward:
+        run_profile_forward(int(args.profile_forward[0]), *args.profile_forward[1:2])
         return
     if args.profile_product:
         run_profile_product(args.profile_product)

@@ -136,6 +136,11 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
   cluster_sync_all();  // barriers initialised and TMEM allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_slot;
+  // The setup above may overlap the kernel before this one (programmatic dependent launch); the
+  // codes and s_x come from it, so wait for it here. The next kernel may then be scheduled onto
+  // the SMs this grid leaves as its clusters finish (it waits for this grid before reading Y).
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs)

@@ -229,9 +229,9 @@ hbl_status run_nq(const void* X, const float* gain, int M, int K, int quant, flo
   a.eps_q = eps_q;
   a.tpr = 0;
   a.rows = 0;
-  // K is a multiple of 256 in [256, 32768], so tpr lands in [32, 1024]
+  // K is a multiple of 256 in [256, 32768], so tpr lands in [32, 1024]; from 4096 features on a
+  // thread keeps four 16-byte loads in flight
   if (K <= 2048) return launch_nq_e<8>(a, quant, stream);
-  if (K <= 16384) return launch_nq_e<16>(a, quant, stream);
   return launch_nq_e<32>(a, quant, stream);
 }
 
@@ -322,10 +322,10 @@ hbl_status run_nfq(const void* X, const float* gain, int M, int K, int had_block
 
 // ---------------------------------------------------------------- products
 
-template <int MT>
+template <int MT, bool FUSED>
 hbl_status launch_decode_t(const DecodeArgs& a, int smem, cudaStream_t s) {
   static SmemLimit lim;
-  cudaError_t e = allow_smem(gemm_decode_kernel<MT>, smem, lim);
+  cudaError_t e = allow_smem(gemm_decode_kernel<MT, FUSED>, smem, lim);
   if (e != cudaSuccess) return cuda_fail(e);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(((a.N + 127) / 128) * a.S, 1, 1);
@@ -341,16 +341,18 @@ hbl_status launch_decode_t(const DecodeArgs& a, int smem, cudaStream_t s) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  e = cudaLaunchKernelEx(&cfg, gemm_decode_kernel<MT>, a);
+  e = cudaLaunchKernelEx(&cfg, gemm_decode_kernel<MT, FUSED>, a);
   if (e != cudaSuccess) return cuda_fail(e);
   HBL_CHECK_LAUNCH();
   return HBL_OK;
 }
 
-// One launch per slice of up to 8 token rows. A cluster of S CTAs splits K for each 128-feature
-// tile: S is chosen so that about two CTAs run per SM, and large enough that the CTA's staged
-// activations stay within 32 KB (next to the 64 KB weight ring).
-hbl_status run_decode(const DecodeArgs& a0, cudaStream_t s) {
+// One launch per slice of up to 8 token rows (fused: up to 4). A cluster of S CTAs splits K for
+// each 128-feature tile: S is chosen so that about two CTAs run per SM, and large enough that the
+// CTA's staged activations stay within 32 KB (next to the 64 KB weight ring). The fused forward
+// takes S down to a power of two, so that K / S is a power of two as well (its slices are blocks
+// of the transform's index space), and adds an fp32 working copy of its slice of the rows.
+hbl_status run_decode(const DecodeArgs& a0, bool fused, cudaStream_t s) {
   DecodeArgs a = a0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -365,15 +367,25 @@ hbl_status run_decode(const DecodeArgs& a0, cudaStream_t s) {
     if (S > 8) S = 8;
     if (S > KB) S = KB;
     if (S < 1) S = 1;
+    if (fused)
+      while (S & (S - 1)) --S;
     a.S = S;
     const int range = (KB + S - 1) / S * 128;
-    const int smem = dec_slot_bytes(S, MT) + kDecRingBytes + MT * range;
+    const int smem = dec_slot_bytes(S, MT) + kDecRingBytes + MT * range + (fused ? MT * range * 4 : 0);
     hbl_status st;
-    switch (MT) {
-      case 1: st = launch_decode_t<1>(a, smem, s); break;
-      case 2: st = launch_decode_t<2>(a, smem, s); break;
-      case 4: st = launch_decode_t<4>(a, smem, s); break;
-      default: st = launch_decode_t<8>(a, smem, s); break;
+    if (fused) {
+      switch (MT) {
+        case 1: st = launch_decode_t<1, true>(a, smem, s); break;
+        case 2: st = launch_decode_t<2, true>(a, smem, s); break;
+        default: st = launch_decode_t<4, true>(a, smem, s); break;
+      }
+    } else {
+      switch (MT) {
+        case 1: st = launch_decode_t<1, false>(a, smem, s); break;
+        case 2: st = launch_decode_t<2, false>(a, smem, s); break;
+        case 4: st = launch_decode_t<4, false>(a, smem, s); break;
+        default: st = launch_decode_t<8, false>(a, smem, s); break;
+      }
     }
     if (st != HBL_OK) return st;
     a.m0 += MT;
@@ -429,9 +441,20 @@ hbl_status run_tc2(const void* codes_i8, const int8_t* w_i8, const TcArgs& a0, c
   const int pairs = device_sms(dev) / 2;
   const int grid = 2 * (ntiles < pairs ? ntiles : pairs);
   static SmemLimit lim;
-  const cudaError_t e = allow_smem(gemm_tc2_kernel, kT2Smem, lim);
+  cudaError_t e = allow_smem(gemm_tc2_kernel, kT2Smem, lim);
   if (e != cudaSuccess) return cuda_fail(e);
-  gemm_tc2_kernel<<<grid, kT2Threads, kT2Smem, s>>>(mA, mB, a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kT2Threads, 1, 1);
+  cfg.dynamicSmemBytes = kT2Smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may overlap the kernel before
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gemm_tc2_kernel, mA, mB, a);
+  if (e != cudaSuccess) return cuda_fail(e);
   HBL_CHECK_LAUNCH();
   return HBL_OK;
 }
@@ -516,6 +539,9 @@ hbl_status run_swap(const void* codes_i8, const void* w2, const TcArgs& t, cudaS
 // codes up to 8 (the tensor-core kernels read one int8 per code).
 constexpr int kDecodeMaxM = 4;
 constexpr int kDecodeMaxMPacked = 8;
+// hbl_forward fuses the activation side into the decode product up to these sizes.
+constexpr int kFusedMaxM = 1;
+constexpr int kFusedMaxK = 8192;
 
 hbl_status run_gemm(const void* codes, int fmt, int abits, const float* s_x, const void* packed, float alpha,
                     int M, int N, int K, void* Y, int out_dtype, int32_t* acc_debug, cudaStream_t s) {
@@ -536,7 +562,13 @@ hbl_status run_gemm(const void* codes, int fmt, int abits, const float* s_x, con
     d.Y = Y;
     d.out_bf16 = out_dtype == HBL_OUT_BF16;
     d.acc_debug = acc_debug;
-    return run_decode(d, s);
+    d.X = nullptr;
+    d.gain = nullptr;
+    d.hb = 1;
+    d.quant = 0;
+    d.eps_norm = 0.f;
+    d.eps_q = 0.f;
+    return run_decode(d, false, s);
   }
   if (packed4) return HBL_EUNSUPPORTED;  // the tensor-core path reads one int8 per code
   TcArgs t;
@@ -856,6 +888,43 @@ hbl_status hbl_forward(const void* X, const float* gain, const void* packed, siz
   if (ws_bytes < hbl_forward_workspace(M, K, quant)) return HBL_EINVAL;
   if (packed_bytes < blob_layout(K, N).total || !aligned(packed, 256) || !aligned(Y, 16)) return HBL_EINVAL;
   const int abits = quant == HBL_Q_A8_ABSMAX ? 8 : 4;
+  // One token (decode) of a power-of-two K up to kFusedMaxK: one launch computes the activation
+  // side of each CTA's slice of K in the product kernel itself (one transform block, blocks of a
+  // power of two, or none); the codes never leave the SM. With more tokens or wider rows every CTA
+  // repeats more of the row's transform than the separate activation kernel costs (measured on
+  // B200, Wo 4096 -> 4096: 8.0 against 9.2 us at one token, 16.1 against 10.8 us at four; Wdown
+  // 16384 -> 4096 at one token: 12.3 against 11.8 us), so those take the two-kernel path.
+  if (M <= kFusedMaxM && K <= kFusedMaxK && is_pow2(K)) {
+    const int n = had_block == 0 ? K : had_block;
+    const bool hb_ok = n == 1 || (is_pow2(n) && n >= 256 && n <= 16384 && (K % n) == 0);
+    if (hb_ok) {
+      if (quant != HBL_Q_A8_ABSMAX && quant != HBL_Q_A4_ABSMEAN && quant != HBL_Q_A4_ABSMAX) return HBL_EUNSUPPORTED;
+      if (!(eps_norm >= 0.f) || !(eps_q >= 0.f)) return HBL_EINVAL;
+      if (!aligned(X, 16) || (gain && !aligned(gain, 4))) return HBL_EINVAL;
+      if (out_dtype != HBL_OUT_F32 && out_dtype != HBL_OUT_BF16) return HBL_EINVAL;
+      const BlobLayout bl = blob_layout(K, N);
+      DecodeArgs d;
+      d.m0 = 0;
+      d.codes = nullptr;
+      d.packed4 = 0;
+      d.s_x = nullptr;
+      d.w2 = reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(packed) + bl.off0);
+      d.alpha = alpha;
+      d.M = M;
+      d.N = N;
+      d.K = K;
+      d.Y = Y;
+      d.out_bf16 = out_dtype == HBL_OUT_BF16;
+      d.acc_debug = nullptr;
+      d.X = static_cast<const uint16_t*>(X);
+      d.gain = gain;
+      d.hb = n;
+      d.quant = (int)quant;
+      d.eps_norm = eps_norm;
+      d.eps_q = eps_q;
+      return run_decode(d, true, reinterpret_cast<cudaStream_t>(stream));
+    }
+  }
   const hbl_codes_fmt fmt = HBL_CODES_I8;  // both tensor-core products read one int8 per code
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* codes = ws;

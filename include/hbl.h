@@ -202,6 +202,11 @@ hbl_status hbl_ternary_gemm(const void* codes, hbl_codes_fmt fmt, int abits, con
 
 /* ---------------------------------------------------------------------------------------
  * The whole layer forward: hbl_norm_fht_quant into `workspace`, then hbl_ternary_gemm.
+ * For one token (M = 1) with K a power of two up to 8192 (had_block 0, 1, or a power of two)
+ * it is one launch instead: the decode product computes the codes of each CTA's slice of K from
+ * the bf16 row itself (the transform's stages across slices as signed sums of the row's slices,
+ * the row statistics reduced over the CTA cluster), and writes nothing to `workspace`. The
+ * result is the same layer, up to the one-step code flips any two fp32 evaluations may differ by.
  *   workspace  device scratch, ws_bytes >= hbl_forward_workspace(M, K, quant), 256-byte aligned
  * Asynchronous. */
 size_t hbl_forward_workspace(int M, int K, hbl_quant quant);

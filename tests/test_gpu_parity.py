@@ -332,6 +332,15 @@ def test_bf16_output():
 
 # ---------------------------------------------------------------- whole layer
 
+def fused_forward(spec):
+    """hbl_forward runs the fused decode kernel (activation side computed in the product) for one
+    token with K a power of two up to 8192: one transform block, blocks of a power of two, or none."""
+    K = spec.K
+    n = K if spec.had_block == 0 else spec.had_block
+    return (spec.M == 1 and K <= 8192 and K & (K - 1) == 0
+            and (n == 1 or (n & (n - 1) == 0 and 256 <= n <= 16384 and K % n == 0)))
+
+
 def check_forward(spec, rows=None, out_dtype=hbl.HBL_OUT_F32):
     """Run hbl_forward on the full spec; compare `rows` (default: all) with the oracle."""
     x = inputs.activations(spec)
@@ -355,16 +364,24 @@ def check_forward(spec, rows=None, out_dtype=hbl.HBL_OUT_F32):
     assert_codes_close(q_gpu, ref["q"])
     np.testing.assert_allclose(s_gpu, ref["s"], rtol=1e-5)
     ys = y[sel]
+    tnorm = np.linalg.norm(ref["t"].astype(np.float64), axis=1)
+    rel = 1e-3 if out_dtype == hbl.HBL_OUT_F32 else 4e-3
+    err = np.linalg.norm(ys - ref["y"], axis=1)
+    if fused_forward(spec):
+        # the product kernel computed its own codes (they never leave the SM): the same one-step
+        # flip budget per row, charged at the largest weight-row norm
+        flips = max(1, int(1e-4 * spec.K))
+        bound = rel * np.linalg.norm(ref["y"], axis=1) + flips * tnorm.max() * ref["s"] * ref["alpha"]
+        assert np.all(err <= bound + 1e-30)
+        return
     # exact product of the GPU's own codes, oracle weights and scales
     y_own = oracle.dequant(oracle.ternary_matmul(q_gpu, ref["t"]), ref["s"], ref["alpha"])
     tol_own = 1e-5 if out_dtype == hbl.HBL_OUT_F32 else 2 ** -8
     assert np.all(row_rel_err(ys, y_own) <= tol_own)
     # end to end against the oracle, with the permitted flips accounted for exactly
     dq = np.abs(q_gpu.astype(np.float64) - ref["q"])
-    tnorm = np.linalg.norm(ref["t"].astype(np.float64), axis=1)
     flip_part = (dq @ tnorm) * ref["s"] * ref["alpha"]
-    err = np.linalg.norm(ys - ref["y"], axis=1)
-    bound = (1e-3 if out_dtype == hbl.HBL_OUT_F32 else 4e-3) * np.linalg.norm(ref["y"], axis=1) + flip_part
+    bound = rel * np.linalg.norm(ref["y"], axis=1) + flip_part
     assert np.all(err <= bound + 1e-30)
 
 
@@ -427,6 +444,45 @@ def test_forward_with_rotated_weights(name, M):
             + np.abs(q_gpu.astype(np.float64)) @ dt.sum(axis=1)) * ref["s"] * ref["alpha"]
     err = np.linalg.norm(y - ref["y"], axis=1)
     assert np.all(err <= 1e-3 * np.linalg.norm(ref["y"], axis=1) + flip + 1e-30)
+
+
+FUSED_CASES = [
+    # (K, N, had_block, M, quant, gain, eps_norm, eps_q)
+    (4096, 4096, 0, 1, hbl.HBL_Q_A4_ABSMEAN, False, 1e-6, 0.0),
+    (8192, 520, 0, 1, hbl.HBL_Q_A8_ABSMAX, True, 1e-6, 0.0),
+    (4096, 4096, 0, 1, hbl.HBL_Q_A4_ABSMAX, False, 1e-2, 1e-3),
+    (4096, 264, 256, 1, hbl.HBL_Q_A4_ABSMEAN, True, 1e-6, 0.0),
+    (8192, 2560, 2048, 1, hbl.HBL_Q_A4_ABSMEAN, False, 1e-6, 0.0),
+    (2048, 2048, 0, 1, hbl.HBL_Q_A8_ABSMAX, False, 1e-6, 1e-3),
+    (256, 256, 0, 1, hbl.HBL_Q_A8_ABSMAX, False, 1e-6, 0.0),
+    (8192, 136, 4096, 1, hbl.HBL_Q_A4_ABSMEAN, False, 1e-6, 0.0),
+    (4096, 12288, 1, 1, hbl.HBL_Q_A4_ABSMEAN, True, 1e-6, 0.0),
+    (1024, 128, 1, 1, hbl.HBL_Q_A8_ABSMAX, False, 1e-6, 0.0),
+]
+
+
+@pytest.mark.parametrize("K,N,had_block,M,quant,use_gain,eps_norm,eps_q", FUSED_CASES)
+def test_fused_decode_forward(K, N, had_block, M, quant, use_gain, eps_norm, eps_q):
+    # one launch per layer for a few tokens: the product kernel computes each CTA's slice of the
+    # activation codes itself (transform stages across slices as signed sums, statistics reduced
+    # over the cluster); compared with the oracle per row with the one-step flip budget
+    abits, mode = QUANT_NAME[quant]
+    spec = spec_like("wdown_7b_a4", K=K, N=N, M=M, had_block=had_block, abits=abits, seed=K + N + M)
+    assert fused_forward(spec)
+    x = inputs.activations(spec)
+    W = inputs.weights(spec)
+    gain = np.random.default_rng(K).uniform(0.5, 1.5, size=K).astype(np.float32) if use_gain else None
+    packed, alpha = hbl.hbl_pack_weights(torch.from_numpy(W).cuda())
+    g = None if gain is None else torch.from_numpy(gain).cuda()
+    Y = hbl.hbl_forward(to_dev_bf16(x), packed, alpha, N, g, had_block, quant, eps_norm, eps_q)
+    torch.cuda.synchronize()
+    y = Y.cpu().numpy()
+    ref = oracle.h_bitlinear_forward(x, W, gain, had_block, abits, mode, eps_norm=eps_norm, eps_q=eps_q)
+    tnorm = np.linalg.norm(ref["t"].astype(np.float64), axis=1)
+    flips = max(1, int(1e-4 * K))
+    bound = 1e-3 * np.linalg.norm(ref["y"], axis=1) + flips * tnorm.max() * ref["s"] * ref["alpha"]
+    err = np.linalg.norm(y - ref["y"], axis=1)
+    assert np.all(err <= bound + 1e-30), (err / np.linalg.norm(ref["y"], axis=1))
 
 
 FULL = [("single_a8_16x256", None), ("wo_1p3b_a4", None), ("wdown_3b_a4", None), ("wo_7b_a4", 8192),
