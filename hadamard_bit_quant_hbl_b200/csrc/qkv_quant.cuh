@@ -10,16 +10,36 @@
 // RoPE is the LLaMA form of the model's LLaMA-like parts ("BitNet v2：原生4位激活"): feature f of a
 // head pairs with f + D/2 and both turn by the angle pos * theta^(-2f/D).
 //
-// Layout: one CTA per token. Its threads first build the cos/sin table of the token's D/2 angles
-// in shared memory (angle formed and reduced modulo 2 pi in fp64, then rounded to fp32), then each
-// warp takes heads in turn: lane l holds features l*E .. l*E+E-1 (E = D/32), whose RoPE partners
-// sit in lane l ^ 16. Codes leave as a little-endian bit string per head (code j at bits
-// [b j, b j + b)), each group of 8 codes (b bytes) assembled across the lanes that hold it.
+// Layout: one CTA per kQkvTokens tokens. Its threads first build the cos/sin table of those
+// tokens' D/2 angles in shared memory together (angle formed and reduced modulo 2 pi in fp64, then
+// rounded to fp32; one barrier), then each warp takes (token, head) pairs in turn: lane l holds
+// features l*E .. l*E+E-1 (E = D/32), whose RoPE partners sit in lane l ^ 16. Codes leave as a
+// little-endian bit string per head (code j at bits [b j, b j + b)), each group of 8 codes
+// (b bytes) assembled across the lanes that hold it.
 #pragma once
 
 #include "common.cuh"
 
 namespace hbl {
+
+constexpr int kQkvTokens = 4;  // tokens per CTA
+
+// Code of one value: u = RoundClip(L (x + gamma) / (2 gamma), 0, L) with mult = (L/2) / gamma.
+// The fused multiply-add gives the value to within a few ulps; only where that lands within
+// 2^-12 of a .5 boundary is the value formed again in fp64 as (L x + L gamma) / (2 gamma), which
+// is exact for bf16 inputs (so that a value exactly on a boundary goes to the even code) and is the
+// expression a float64 evaluation of the reading uses.
+template <int BITS>
+__device__ __forceinline__ float unsigned_code(float x, float g, float mult) {
+  constexpr float kL = (float)((1 << BITS) - 1);
+  float t = fmaf(x, mult, 0.5f * kL);
+  const float fr = t - floorf(t);
+  if (fabsf(fr - 0.5f) < 2.44140625e-4f) {  // 2^-12
+    const double L = (double)kL, xd = (double)x, gd = (double)g;
+    t = gd > 0.0 ? (float)rint((L * xd + L * gd) / (2.0 * gd)) : rintf(0.5f * kL);
+  }
+  return fminf(fmaxf(rintf(t), 0.f), kL);
+}
 
 struct QkvArgs {
   const uint16_t* X;  // bf16; token m, head h at X + m * row_stride + h * D
@@ -76,39 +96,40 @@ __global__ void __launch_bounds__(256) qkv_quant_kernel(QkvArgs a) {
   constexpr float kL = (float)((1 << BITS) - 1);
   constexpr int LPG = 8 / E;  // lanes holding one group of 8 codes
   constexpr int HEAD_BYTES = D * BITS / 8;
-  __shared__ float cs[HALF], sn[HALF];
+  __shared__ float cs[kQkvTokens][HALF], sn[kQkvTokens][HALF];
 
-  const int m = blockIdx.x;
+  const int m0 = blockIdx.x * kQkvTokens;
+  const int nt = a.M - m0 < kQkvTokens ? a.M - m0 : kQkvTokens;
   // X may come from the kernel before this one (programmatic dependent launch)
   pdl_wait();
   pdl_launch_dependents();
   if constexpr (ROPE) {
     const double two_pi = 6.283185307179586476925;
     const double lt = log((double)a.theta);
-    const double p = (double)a.pos[m];
-    for (int f = threadIdx.x; f < HALF; f += blockDim.x) {
-      const double ang = p * exp(-2.0 * (double)f / (double)D * lt);
+    for (int e = threadIdx.x; e < nt * HALF; e += blockDim.x) {
+      const int t = e / HALF, f = e - t * HALF;
+      const double ang = (double)a.pos[m0 + t] * exp(-2.0 * (double)f / (double)D * lt);
       const double r = ang - two_pi * rint(ang / two_pi);
       double s, c;
       sincos(r, &s, &c);
-      cs[f] = (float)c;
-      sn[f] = (float)s;
+      cs[t][f] = (float)c;
+      sn[t][f] = (float)s;
     }
     __syncthreads();
   }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const uint16_t* xrow = a.X + (size_t)m * a.row_stride;
-  for (int h = warp; h < a.H; h += nwarps) {
-    float v[E];
-    qkv_load<E>(xrow + (size_t)h * D + lane * E, v);
+  // one (token, head) pair: rotate, absmax, codes, pack, store
+  auto head = [&](int th, float (&v)[E]) {
+    const int t = th / a.H, h = th - t * a.H;
+    const int m = m0 + t;
     if constexpr (ROPE) {
       const bool first = lane < 16;
 #pragma unroll
       for (int e = 0; e < E; ++e) {
         const float partner = __shfl_xor_sync(0xffffffffu, v[e], 16);
         const int f = (lane & 15) * E + e;
-        const float c = cs[f], s = sn[f];
-        v[e] = first ? fmaf(v[e], c, -partner * s) : fmaf(partner, s, v[e] * c);
+        const float c = cs[t][f], sn_ = sn[t][f];
+        v[e] = first ? fmaf(v[e], c, -partner * sn_) : fmaf(partner, sn_, v[e] * c);
       }
     }
     float g = 0.f;
@@ -116,15 +137,11 @@ __global__ void __launch_bounds__(256) qkv_quant_kernel(QkvArgs a) {
     for (int e = 0; e < E; ++e) g = fmaxf(g, fabsf(v[e]));
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, o));
-    // u = rint(L (x + gamma) / (2 gamma)): the numerator by one fused multiply-add (exact for bf16
-    // inputs, whose products with L need 16 bits), then a correctly rounded division, so that a
-    // value exactly on a .5 boundary stays on it and goes to the even code
-    const float lg = kL * g, den = 2.f * g;
+    const float mult = g > 0.f ? 0.5f * kL / g : 0.f;
     unsigned long long bits = 0;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-      const float t = g > 0.f ? __fdiv_rn(fmaf(kL, v[e], lg), den) : 0.5f * kL;
-      const float q = fminf(fmaxf(rintf(t), 0.f), kL);
+      const float q = unsigned_code<BITS>(v[e], g, mult);
       bits |= (unsigned long long)(uint32_t)q << (((lane % LPG) * E + e) * BITS);
     }
 #pragma unroll
@@ -132,6 +149,20 @@ __global__ void __launch_bounds__(256) qkv_quant_kernel(QkvArgs a) {
     const size_t mh = (size_t)m * a.H + h;
     if (lane % LPG == 0) qkv_store_group<BITS>(a.codes + mh * HEAD_BYTES + (lane / LPG) * BITS, bits);
     if (lane == 0) a.gamma[mh] = g;
+  };
+  auto src = [&](int th) {
+    const int t = th / a.H, h = th - t * a.H;
+    return a.X + (size_t)(m0 + t) * a.row_stride + (size_t)h * D + lane * E;
+  };
+  // two pairs per step, both loads issued before either is used
+  const int npairs = nt * a.H;
+  for (int th0 = warp; th0 < npairs; th0 += 2 * nwarps) {
+    const int th1 = th0 + nwarps;
+    float v0[E], v1[E];
+    qkv_load<E>(src(th0), v0);
+    if (th1 < npairs) qkv_load<E>(src(th1), v1);
+    head(th0, v0);
+    if (th1 < npairs) head(th1, v1);
   }
 }
 
