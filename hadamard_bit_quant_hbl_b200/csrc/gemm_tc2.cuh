@@ -283,4 +283,217 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
   }
 }
 
+// ---------------------------------------------------------------- split-K over two SM pairs
+//
+// For token counts whose 256 x 256 tiles would leave half the SM pairs idle (M = 512 at N = 4096
+// gives 32 tiles for 74 pairs), a cluster of four CTAs (two SM pairs) computes one tile: pair p
+// accumulates the k-blocks [KB p / 2, KB (p + 1) / 2) in its own tensor memory, exactly as above.
+// Then pair 1 writes its int32 partial sums into the shared memory of the matching CTA of pair 0
+// (distributed shared memory; the rings are idle by then), and pair 0 adds them to its own in the
+// epilogue. Integer sums: the result is bit-identical to the one-pair kernel's.
+constexpr int kT2sRed = 128 * kT2BN * 4;  // bytes of one CTA's partial sums (128 rows x 256 int32)
+static_assert(kT2sRed <= kT2Stages * (kT2StageA + kT2StageB), "partial sums fit in the ring");
+
+__global__ void __launch_bounds__(kT2Threads, 1)
+gemm_tc2s_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                 const Tc2Args a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw2s[];
+  __shared__ __align__(8) uint64_t full_bar[kT2Stages], empty_bar[kT2Stages];
+  __shared__ __align__(8) uint64_t accf_bar, drain_bar;
+  __shared__ uint32_t tmem_base_slot;
+  __shared__ volatile int abort_flag;
+
+  uint8_t* smem = align_shared<1024>(smem_raw2s);
+  uint8_t* smA = smem;
+  uint8_t* smB = smem + kT2Stages * kT2StageA;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();      // 0..3
+  const uint32_t pair = rank >> 1, r = rank & 1;
+  const uint32_t lead = rank & ~1u;             // the pair's leader
+  const bool leader = r == 0;
+  const int t = blockIdx.x >> 2;                // one tile per cluster
+  const int tm = t / a.tiles_n, tn = t - tm * a.tiles_n;
+  const int KB = a.K / kT2BK;
+  const int kb0 = (int)(pair * KB / 2), kb1 = (int)((pair + 1) * KB / 2);
+  const uint16_t pair_mask = (uint16_t)(0x3u << (2 * pair));
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int st = 0; st < kT2Stages; ++st) {
+      mbar_init(&full_bar[st], 1);
+      mbar_init(&empty_bar[st], 1);
+    }
+    mbar_init(&accf_bar, 1);
+    mbar_init(&drain_bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    tma_prefetch_desc(&mapA);
+    tma_prefetch_desc(&mapB);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], 256;"
+                 ::"r"(smem_u32(&tmem_base_slot)) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();  // barriers initialised and TMEM allocated in all four CTAs
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_slot;
+  pdl_wait();  // the codes and s_x come from the kernel before this one
+  pdl_launch_dependents();
+
+  bool ok = true;
+  if (warp == 0) {
+    // ---------------- TMA producer (every CTA): its halves of the pair's k-blocks
+    if (lane == 0) {
+      const uint32_t full0_leader = mapa_shared(smem_u32(&full_bar[0]), lead);
+      const int rowA = tm * kT2BM + (int)r * 128;
+      const int rowB = tn * kT2BN + (int)r * 128;
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag)) break;
+        if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2u * (kT2StageA + kT2StageB));
+        const uint32_t fb = full0_leader + (uint32_t)(stage * sizeof(uint64_t));
+        tma_load_2d_pair(smA + stage * kT2StageA, &mapA, fb, kb * kT2BK, rowA);
+        tma_load_2d_pair(smB + stage * kT2StageB, &mapB, fb, kb * kT2BK, rowB);
+        if (++stage == kT2Stages) { stage = 0; phase ^= 1u; }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (the pair's leader)
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(kT2BM, kT2BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool any = false;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(&full_bar[stage], phase, &abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smA + stage * kT2StageA);
+        const uint32_t b_addr = smem_u32(smB + stage * kT2StageB);
+#pragma unroll
+        for (int kk = 0; kk < kT2BK / 32; ++kk)
+          mma_i8_pair(tmem_base, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32), idesc,
+                      (kb > kb0 || kk) ? 1u : 0u);
+        any = true;
+        asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                     ::"r"(smem_u32(&empty_bar[stage])), "h"(pair_mask) : "memory");
+        if (++stage == kT2Stages) { stage = 0; phase ^= 1u; }
+      }
+      if (ok) {
+        asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                     ::"r"(smem_u32(&accf_bar)), "h"(pair_mask) : "memory");
+      } else if (any) {
+        asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                     ::"r"(smem_u32(&drain_bar)) : "memory");
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&drain_bar, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  }
+
+  // ---------------- the pair's sum is complete in its tensor memory (epilogue warps 2..5, TMEM
+  // lane quarter warp % 4: rows 32 q .. 32 q + 31 of this CTA's 128)
+  const int q = warp & 3;
+  int acc_ok = 1;
+  if (warp >= 2) {
+    if (lane == 0) acc_ok = mbar_wait(&accf_bar, 0, &abort_flag) ? 1 : 0;
+    acc_ok = __shfl_sync(0xffffffffu, acc_ok, 0);
+    tc_fence_after();
+  }
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();  // both pairs' main loops are done: every ring is idle
+  tc_fence_after();
+  const int lrow = q * 32 + lane;  // row within this CTA's 128
+  int32_t* red = reinterpret_cast<int32_t*>(smem);  // [128 rows][256] partial sums of pair 1
+  if (warp >= 2 && pair == 1) {
+    // pair 1: partial sums into the matching CTA of pair 0, row-major int32
+    const uint32_t dst0 = mapa_shared(smem_u32(red), rank - 2);
+#pragma unroll 1
+    for (int c = 0; c < kT2BN / 32; ++c) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), v);
+      if (!acc_ok) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = 0u;
+      }
+      const uint32_t dst = dst0 + (uint32_t)((lrow * kT2BN + c * 32) * 4);
+#pragma unroll
+      for (int j = 0; j < 32; j += 4)
+        asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};"
+                     ::"r"(dst + (uint32_t)(j * 4)), "r"(v[j]), "r"(v[j + 1]), "r"(v[j + 2]), "r"(v[j + 3]) : "memory");
+    }
+  }
+  tc_fence_before();
+  cluster_sync_all();  // pair 1's partial sums have landed in pair 0
+  tc_fence_after();
+  if (warp >= 2 && pair == 0) {
+    const int row = tm * kT2BM + (int)r * 128 + lrow;
+    const bool rok = row < a.M;
+    const float scale = rok ? a.s_x[row] * a.alpha : 0.f;
+#pragma unroll 1
+    for (int c = 0; c < kT2BN / 32; ++c) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), v);
+      const int col0 = tn * kT2BN + c * 32;
+      if (!rok || col0 >= a.N) continue;
+      const int32_t* pr = red + lrow * kT2BN + c * 32;
+      int32_t s32[32];
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        const int4 p4 = *reinterpret_cast<const int4*>(pr + j);
+        s32[j] = (acc_ok ? (int32_t)v[j] : 0) + p4.x;
+        s32[j + 1] = (acc_ok ? (int32_t)v[j + 1] : 0) + p4.y;
+        s32[j + 2] = (acc_ok ? (int32_t)v[j + 2] : 0) + p4.z;
+        s32[j + 3] = (acc_ok ? (int32_t)v[j + 3] : 0) + p4.w;
+      }
+      const bool full = col0 + 32 <= a.N;
+      if (a.out_bf16) {
+        __nv_bfloat16* yrow = reinterpret_cast<__nv_bfloat16*>(a.Y) + (size_t)row * a.N + col0;
+        if (full) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            uint4 o;
+            uint32_t* op = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const __nv_bfloat162 p2 = __floats2bfloat162_rn((float)s32[j + 2 * h] * scale,
+                                                             (float)s32[j + 2 * h + 1] * scale);
+              op[h] = *reinterpret_cast<const uint32_t*>(&p2);
+            }
+            *reinterpret_cast<uint4*>(yrow + j) = o;
+          }
+        } else {
+          for (int j = 0; j < 32 && col0 + j < a.N; ++j) yrow[j] = __float2bfloat16_rn((float)s32[j] * scale);
+        }
+      } else {
+        float* yrow = reinterpret_cast<float*>(a.Y) + (size_t)row * a.N + col0;
+        if (full) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(yrow + j) = make_float4((float)s32[j] * scale, (float)s32[j + 1] * scale,
+                                                               (float)s32[j + 2] * scale, (float)s32[j + 3] * scale);
+        } else {
+          for (int j = 0; j < 32 && col0 + j < a.N; ++j) yrow[j] = (float)s32[j] * scale;
+        }
+      }
+      if (a.acc_debug) {
+        int32_t* drow = a.acc_debug + (size_t)row * a.N + col0;
+        for (int j = 0; j < 32 && col0 + j < a.N; ++j) drow[j] = s32[j];
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, 256;" ::"r"(tmem_base) : "memory");
+  }
+}
+
 }  // namespace hbl

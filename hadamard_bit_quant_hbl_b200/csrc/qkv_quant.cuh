@@ -18,6 +18,8 @@
 // (b bytes) assembled across the lanes that hold it.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace hbl {
@@ -30,15 +32,15 @@ constexpr int kQkvTokens = 4;  // tokens per CTA
 // is exact for bf16 inputs (so that a value exactly on a boundary goes to the even code) and is the
 // expression a float64 evaluation of the reading uses.
 template <int BITS>
-__device__ __forceinline__ float unsigned_code(float x, float g, float mult) {
+__device__ __forceinline__ uint32_t unsigned_code(float x, float g, float mult) {
   constexpr float kL = (float)((1 << BITS) - 1);
-  float t = fmaf(x, mult, 0.5f * kL);
-  const float fr = t - floorf(t);
-  if (fabsf(fr - 0.5f) < 2.44140625e-4f) {  // 2^-12
+  const float t = fmaf(x, mult, 0.5f * kL);
+  float q = rintf(t);
+  if (fabsf(t - q) > 0.5f - 2.44140625e-4f) {  // within 2^-12 of a boundary
     const double L = (double)kL, xd = (double)x, gd = (double)g;
-    t = gd > 0.0 ? (float)rint((L * xd + L * gd) / (2.0 * gd)) : rintf(0.5f * kL);
+    q = gd > 0.0 ? (float)rint((L * xd + L * gd) / (2.0 * gd)) : rintf(0.5f * kL);
   }
-  return fminf(fmaxf(rintf(t), 0.f), kL);
+  return (uint32_t)fminf(fmaxf(q, 0.f), kL);
 }
 
 struct QkvArgs {
@@ -96,7 +98,7 @@ __global__ void __launch_bounds__(256) qkv_quant_kernel(QkvArgs a) {
   constexpr float kL = (float)((1 << BITS) - 1);
   constexpr int LPG = 8 / E;  // lanes holding one group of 8 codes
   constexpr int HEAD_BYTES = D * BITS / 8;
-  __shared__ float cs[kQkvTokens][HALF], sn[kQkvTokens][HALF];
+  __shared__ float cs[kQkvTokens][HALF], sin_tab[kQkvTokens][HALF];
 
   const int m0 = blockIdx.x * kQkvTokens;
   const int nt = a.M - m0 < kQkvTokens ? a.M - m0 : kQkvTokens;
@@ -113,56 +115,63 @@ __global__ void __launch_bounds__(256) qkv_quant_kernel(QkvArgs a) {
       double s, c;
       sincos(r, &s, &c);
       cs[t][f] = (float)c;
-      sn[t][f] = (float)s;
+      sin_tab[t][f] = (float)s;
     }
     __syncthreads();
   }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  // one (token, head) pair: rotate, absmax, codes, pack, store
-  auto head = [&](int th, float (&v)[E]) {
-    const int t = th / a.H, h = th - t * a.H;
+  // codes of a group of 8 fit 32 bits up to 4 bits per code
+  using Bits = typename std::conditional<(8 * BITS <= 32), uint32_t, unsigned long long>::type;
+  const bool first = lane < 16;
+  for (int t = 0; t < nt; ++t) {
     const int m = m0 + t;
+    // this lane's angles for the token: the same for every head
+    float c[E], sn[E];
     if constexpr (ROPE) {
-      const bool first = lane < 16;
 #pragma unroll
       for (int e = 0; e < E; ++e) {
-        const float partner = __shfl_xor_sync(0xffffffffu, v[e], 16);
         const int f = (lane & 15) * E + e;
-        const float c = cs[t][f], sn_ = sn[t][f];
-        v[e] = first ? fmaf(v[e], c, -partner * sn_) : fmaf(partner, sn_, v[e] * c);
+        c[e] = cs[t][f];
+        sn[e] = sin_tab[t][f];
       }
     }
-    float g = 0.f;
+    // up to four heads of this warp in flight: every load issued before the first is used
+    for (int h0 = warp; h0 < a.H; h0 += 4 * nwarps) {
+      float v[4][E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) g = fmaxf(g, fabsf(v[e]));
+      for (int i = 0; i < 4; ++i) {
+        const int h = h0 + i * nwarps;
+        if (h < a.H) qkv_load<E>(a.X + (size_t)m * a.row_stride + (size_t)h * D + lane * E, v[i]);
+      }
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, o));
-    const float mult = g > 0.f ? 0.5f * kL / g : 0.f;
-    unsigned long long bits = 0;
+      for (int i = 0; i < 4; ++i) {
+        const int h = h0 + i * nwarps;
+        if (h >= a.H) break;  // the same in every lane
+        if constexpr (ROPE) {
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const float q = unsigned_code<BITS>(v[e], g, mult);
-      bits |= (unsigned long long)(uint32_t)q << (((lane % LPG) * E + e) * BITS);
+          for (int e = 0; e < E; ++e) {
+            const float partner = __shfl_xor_sync(0xffffffffu, v[i][e], 16);
+            v[i][e] = first ? fmaf(v[i][e], c[e], -partner * sn[e]) : fmaf(partner, sn[e], v[i][e] * c[e]);
+          }
+        }
+        float g = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) g = fmaxf(g, fabsf(v[i][e]));
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, o));
+        const float mult = g > 0.f ? 0.5f * kL / g : 0.f;
+        Bits bits = 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+          bits |= (Bits)unsigned_code<BITS>(v[i][e], g, mult) << (((lane % LPG) * E + e) * BITS);
+#pragma unroll
+        for (int o = 1; o < LPG; o <<= 1) bits |= __shfl_xor_sync(0xffffffffu, bits, o);
+        const size_t mh = (size_t)m * a.H + h;
+        if (lane % LPG == 0)
+          qkv_store_group<BITS>(a.codes + mh * HEAD_BYTES + (lane / LPG) * BITS, (uint64_t)bits);
+        if (lane == 0) a.gamma[mh] = g;
+      }
     }
-#pragma unroll
-    for (int o = 1; o < LPG; o <<= 1) bits |= __shfl_xor_sync(0xffffffffu, bits, o);
-    const size_t mh = (size_t)m * a.H + h;
-    if (lane % LPG == 0) qkv_store_group<BITS>(a.codes + mh * HEAD_BYTES + (lane / LPG) * BITS, bits);
-    if (lane == 0) a.gamma[mh] = g;
-  };
-  auto src = [&](int th) {
-    const int t = th / a.H, h = th - t * a.H;
-    return a.X + (size_t)(m0 + t) * a.row_stride + (size_t)h * D + lane * E;
-  };
-  // two pairs per step, both loads issued before either is used
-  const int npairs = nt * a.H;
-  for (int th0 = warp; th0 < npairs; th0 += 2 * nwarps) {
-    const int th1 = th0 + nwarps;
-    float v0[E], v1[E];
-    qkv_load<E>(src(th0), v0);
-    if (th1 < npairs) qkv_load<E>(src(th1), v1);
-    head(th0, v0);
-    if (th1 < npairs) head(th1, v1);
   }
 }
 

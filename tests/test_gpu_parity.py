@@ -286,6 +286,10 @@ GEMM_CASES = [
     # two TMEM accumulators (80 and 160 tiles for 74 pairs)
     (2560, 512, 2048, 4, hbl.HBL_CODES_I8),
     (2560, 256, 4096, 8, hbl.HBL_CODES_I8),
+    # few tiles over a long K: two SM pairs per tile, the second pair's partial sums added through
+    # distributed shared memory (ragged rows and columns)
+    (512, 16384, 1032, 4, hbl.HBL_CODES_I8),
+    (700, 8192, 264, 8, hbl.HBL_CODES_I8),
 ]
 
 
