@@ -330,7 +330,11 @@ def quantize_unsigned_absmax(x: np.ndarray, bits: int) -> tuple[np.ndarray, np.n
 
 
 def dequantize_unsigned(u: np.ndarray, gamma: np.ndarray, bits: int) -> np.ndarray:
-    """x~ = (2u - (2^b - 1)) * gamma / (2^b - 1) (reading R9)."""
+    """x~ = (2u - (2^b - 1)) * gamma / (2^b - 1) (reading R9).
+
+    Pinned by test_unsigned_quantiser_properties (dequantised values within half a step of x) and
+    test_unsigned_quantiser_closed_form (the b = 3 levels, a zero head dequantising to 0).
+    """
     L = (1 << bits) - 1
     return (2.0 * np.asarray(u, dtype=np.float64) - L) * np.asarray(gamma, dtype=np.float64)[..., None] / L
 
@@ -338,7 +342,10 @@ def dequantize_unsigned(u: np.ndarray, gamma: np.ndarray, bits: int) -> np.ndarr
 def qkv_quant(x: np.ndarray, pos: np.ndarray | None, bits: int, theta: float = 10000.0
               ) -> tuple[np.ndarray, np.ndarray]:
     """RoPE (when pos is given: the Q and K states; V takes none) then per-head unsigned absmax
-    quantisation of x [M, H, D] (float64 values or bf16 bit patterns). Returns (u, gamma)."""
+    quantisation of x [M, H, D] (float64 values or bf16 bit patterns). Returns (u, gamma).
+
+    Pinned through its parts (the rope and quantiser pins above) and bf16_to_f64's pins.
+    """
     if x.dtype == np.uint16:
         x = bf16_to_f64(x)
     if pos is not None:
