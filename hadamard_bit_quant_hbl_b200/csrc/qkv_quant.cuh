@@ -27,20 +27,24 @@ namespace hbl {
 constexpr int kQkvTokens = 4;  // tokens per CTA
 
 // Code of one value: u = RoundClip(L (x + gamma) / (2 gamma), 0, L) with mult = (L/2) / gamma.
-// The fused multiply-add gives the value to within a few ulps; only where that lands within
-// 2^-12 of a .5 boundary is the value formed again in fp64 as (L x + L gamma) / (2 gamma), which
-// is exact for bf16 inputs (so that a value exactly on a boundary goes to the even code) and is the
-// expression a float64 evaluation of the reading uses.
+// t = x mult + L/2 lies in [0, L] up to rounding (|x| <= gamma), so its nearest integer needs no
+// clamp; adding 1.5 * 2^23 rounds it (ties to even) into the low mantissa bits, which are the
+// code. Only where t lands within 2^-12 of a .5 boundary is the value formed again in fp64 as
+// (L x + L gamma) / (2 gamma), which is exact for bf16 inputs (so that a value exactly on a
+// boundary goes to the even code) and is the expression a float64 evaluation of the reading uses.
 template <int BITS>
 __device__ __forceinline__ uint32_t unsigned_code(float x, float g, float mult) {
   constexpr float kL = (float)((1 << BITS) - 1);
+  constexpr float kMagic = 12582912.f;  // 1.5 * 2^23
   const float t = fmaf(x, mult, 0.5f * kL);
-  float q = rintf(t);
-  if (fabsf(t - q) > 0.5f - 2.44140625e-4f) {  // within 2^-12 of a boundary
+  const float y = t + kMagic;
+  uint32_t q = __float_as_uint(y) & 0xffu;
+  if (fabsf(t - (y - kMagic)) > 0.5f - 2.44140625e-4f) {  // within 2^-12 of a boundary
     const double L = (double)kL, xd = (double)x, gd = (double)g;
-    q = gd > 0.0 ? (float)rint((L * xd + L * gd) / (2.0 * gd)) : rintf(0.5f * kL);
+    const double u = gd > 0.0 ? rint((L * xd + L * gd) / (2.0 * gd)) : rint(0.5 * (double)kL);
+    q = (uint32_t)fmin(fmax(u, 0.0), (double)kL);
   }
-  return (uint32_t)fminf(fmaxf(q, 0.f), kL);
+  return q;
 }
 
 struct QkvArgs {
@@ -125,14 +129,15 @@ __global__ void __launch_bounds__(256) qkv_quant_kernel(QkvArgs a) {
   const bool first = lane < 16;
   for (int t = 0; t < nt; ++t) {
     const int m = m0 + t;
-    // this lane's angles for the token: the same for every head
+    // this lane's angles for the token, the same for every head; the first half of a head turns
+    // by -sin against its partner, the second by +sin: x' = x c + partner s' with s' = -+ sin
     float c[E], sn[E];
     if constexpr (ROPE) {
 #pragma unroll
       for (int e = 0; e < E; ++e) {
         const int f = (lane & 15) * E + e;
         c[e] = cs[t][f];
-        sn[e] = sin_tab[t][f];
+        sn[e] = first ? -sin_tab[t][f] : sin_tab[t][f];
       }
     }
     // up to four heads of this warp in flight: every load issued before the first is used
@@ -151,7 +156,7 @@ __global__ void __launch_bounds__(256) qkv_quant_kernel(QkvArgs a) {
 #pragma unroll
           for (int e = 0; e < E; ++e) {
             const float partner = __shfl_xor_sync(0xffffffffu, v[i][e], 16);
-            v[i][e] = first ? fmaf(v[i][e], c[e], -partner * sn[e]) : fmaf(partner, sn[e], v[i][e] * c[e]);
+            v[i][e] = fmaf(partner, sn[e], v[i][e] * c[e]);
           }
         }
         float g = 0.f;

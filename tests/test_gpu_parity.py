@@ -178,13 +178,16 @@ def test_norm_fht_quant_degenerate_rows(K, fmt):
         np.testing.assert_allclose(s[1:], s_ref[1:], rtol=1e-5)
 
 
-def test_norm_fht_quant_eps_q_and_eps_norm():
-    spec = spec_like("wo_1p3b_a4", M=13)
+@pytest.mark.parametrize("K,had_block", [(2048, 0), (4096, 0), (8192, 0), (16384, 0), (11008, 256)])
+def test_norm_fht_quant_eps_q_and_eps_norm(K, had_block):
+    # eps under the RMS root and in the quantiser's divisor, on the CUDA-core kernel (2048) and on
+    # every tensor-core form (one block of 4096 / 8192 / 16384, blocks of 256)
+    spec = spec_like("wo_7b_a4", K=K, M=13, had_block=had_block, seed=K + 5)
     x = inputs.activations(spec)
     for quant in QUANT_NAME:
         abits, mode = QUANT_NAME[quant]
-        q_ref, s_ref = oracle.norm_fht_quant(x, None, 0, abits, mode, eps_norm=1e-2, eps_q=1e-3)
-        q, s = gpu_codes(x, None, 0, quant, hbl.HBL_CODES_I8, eps_norm=1e-2, eps_q=1e-3)
+        q_ref, s_ref = oracle.norm_fht_quant(x, None, had_block, abits, mode, eps_norm=1e-2, eps_q=1e-3)
+        q, s = gpu_codes(x, None, had_block, quant, hbl.HBL_CODES_I8, eps_norm=1e-2, eps_q=1e-3)
         assert_codes_close(q, q_ref)
         np.testing.assert_allclose(s, s_ref, rtol=1e-5)
 
