@@ -513,16 +513,32 @@ hbl_status run_swap(const void* codes_i8, const void* w2, const TcArgs& t, cudaS
   a.N = t.N;
   a.K = t.K;
   a.Mt = (t.M + 15) / 16 * 16;
-  // batches of B k-blocks (fewer for wide activation tiles); shared memory: 2 batch stages of
-  // widened tiles (B x 16 KB each), 2 of 2-bit tiles (B x 4 KB), the rest activation copies of
-  // one batch each (B x Mt x 128 bytes)
-  a.B = a.Mt <= 32 ? 4 : (a.Mt <= 128 ? 2 : 1);
-  a.NA = (kSwSmem - a.B * (kSwNWB * kSwWide + kSwNR * kSwRaw)) / (a.B * a.Mt * kSwBK);
+  // batches of BK k-blocks; tensor memory: nis accumulators of Mt columns, then NS slots of
+  // BK x 32 columns of widened weights; shared memory: NA activation copies of one batch
+  // (BK x Mt x 128 bytes) and NR 2-bit copies (BK x 4 KB). Up to 64 tokens two threads issue the
+  // MMAs (alternate batches, one accumulator each): there an MMA is short and one issuing thread
+  // was the limit; above, two accumulators would leave too few slots.
+  const int BK = a.Mt <= 128 ? 4 : 2;
+  a.nis = a.Mt <= 64 ? 2 : 1;
+  int stride = 16;
+  while (stride < a.Mt) stride *= 2;
+  a.acc_stride = stride;
+  a.acc_cols = a.nis * stride < 32 ? 32 : a.nis * stride;
+  a.NS = (kSwTmemCols - a.acc_cols) / (BK * 32);
+  if (a.NS > kSwMaxNS) a.NS = kSwMaxNS;
+  a.NS -= a.NS % a.nis;  // an issuer's slots (and stages, below) repeat with period nis
+  const int act_stage = BK * a.Mt * kSwBK, raw_stage = BK * kSwRaw;
+  a.NA = (kSwSmem - 4 * raw_stage) / act_stage;
   if (a.NA > kSwMaxNA) a.NA = kSwMaxNA;
   if (a.NA < 1) return HBL_EUNSUPPORTED;  // not reached for Mt <= 256
-  int cols = 32;
-  while (cols < a.Mt) cols *= 2;
-  a.tmem_cols = cols;
+  a.NR = (kSwSmem - a.NA * act_stage) / raw_stage;
+  if (a.NR > kSwMaxNR) a.NR = kSwMaxNR;
+  // a widening warp takes every kSwW-th batch: with NR a multiple of kSwW, the warp that waits for
+  // a ring stage's copy is the one that consumed the stage's previous copy, and with NS >= kSwW
+  // no warp runs two phases ahead on a tensor-memory slot (a parity wait cannot alias)
+  a.NR -= a.NR % kSwW;
+  a.NA -= a.NA % a.nis;
+  if (a.NS < kSwW || a.NR < kSwW || a.NA < 1) return HBL_EUNSUPPORTED;  // not reached for Mt <= 256
   a.Y = t.Y;
   a.out_bf16 = t.out_bf16;
   a.acc_debug = t.acc_debug;
@@ -537,10 +553,11 @@ hbl_status run_swap(const void* codes_i8, const void* w2, const TcArgs& t, cudaS
   a.S = S;
   a.w2 = static_cast<const uint32_t*>(w2);
   CUtensorMap mA;
-  if (!make_map_i8_blocks(&mA, codes_i8, a.K, a.M, a.Mt, a.B)) return HBL_ECUDA;
-  static SmemLimit lim;
+  if (!make_map_i8_blocks(&mA, codes_i8, a.K, a.M, a.Mt, BK)) return HBL_ECUDA;
+  static SmemLimit lim4, lim2;
   const int smem = kSwSmem + 1024;  // + alignment slack
-  cudaError_t e = allow_smem(gemm_swap_kernel, smem, lim);
+  auto kern = BK == 4 ? gemm_swap_kernel<4> : gemm_swap_kernel<2>;
+  cudaError_t e = allow_smem(kern, smem, BK == 4 ? lim4 : lim2);
   if (e != cudaSuccess) return cuda_fail(e);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ntiles * S, 1, 1);
@@ -556,7 +573,7 @@ hbl_status run_swap(const void* codes_i8, const void* w2, const TcArgs& t, cudaS
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  e = cudaLaunchKernelEx(&cfg, gemm_swap_kernel, mA, a);
+  e = cudaLaunchKernelEx(&cfg, kern, mA, a);
   if (e != cudaSuccess) return cuda_fail(e);
   HBL_CHECK_LAUNCH();
   return HBL_OK;

@@ -285,6 +285,11 @@ GEMM_CASES = [
     (300, 2048, 520, 4, hbl.HBL_CODES_I8),
     (257, 11008, 264, 4, hbl.HBL_CODES_I8),
     (200, 4096, 1032, 8, hbl.HBL_CODES_I8),
+    # swapped tiles over a long K: several batches per CTA, so that every ring and tensor-memory
+    # slot wraps (16, 112 and 256 padded tokens)
+    (16, 16384, 4096, 4, hbl.HBL_CODES_I8),
+    (100, 16384, 1024, 8, hbl.HBL_CODES_I8),
+    (256, 16384, 256, 4, hbl.HBL_CODES_I8),
     # more 256 x 256 pair tiles than SM pairs: clusters walk two or more tiles, alternating their
     # two TMEM accumulators (80 and 160 tiles for 74 pairs)
     (2560, 512, 2048, 4, hbl.HBL_CODES_I8),
