@@ -170,4 +170,17 @@ __host__ __device__ constexpr int ilog2_c(int v) { return v <= 1 ? 0 : 1 + ilog2
 
 __host__ __device__ constexpr size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Position in a ring of n stages: the stage and the parity of its current phase.
+struct RingPos {
+  int s = 0;
+  uint32_t ph = 0;
+  __device__ __forceinline__ void advance(int step, int n) {  // step <= n
+    s += step;
+    if (s >= n) {
+      s -= n;
+      ph ^= 1u;
+    }
+  }
+};
+
 }  // namespace hbl

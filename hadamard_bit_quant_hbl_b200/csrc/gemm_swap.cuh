@@ -141,19 +141,6 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// Position in a ring of n stages: the stage and the parity of its current phase.
-struct RingPos {
-  int s = 0;
-  uint32_t ph = 0;
-  __device__ __forceinline__ void advance(int step, int n) {  // step <= n
-    s += step;
-    if (s >= n) {
-      s -= n;
-      ph ^= 1u;
-    }
-  }
-};
-
 template <int BK>
 __global__ void __launch_bounds__(kSwThreads, 1)
 gemm_swap_kernel(const __grid_constant__ CUtensorMap mapA, const SwapArgs a) {

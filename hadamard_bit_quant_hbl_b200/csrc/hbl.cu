@@ -17,6 +17,7 @@
 #include "gemm_swap.cuh"
 #include "norm_fht_quant.cuh"
 #include "norm_fht_quant_tc.cuh"
+#include "norm_fht_quant_tc2.cuh"
 #include "norm_quant.cuh"
 #include "pack_weights.cuh"
 #include "qkv_quant.cuh"
@@ -181,6 +182,32 @@ hbl_status launch_nfq_tc(const NfqArgs& a, cudaStream_t s) {
   return HBL_OK;
 }
 
+template <int QM, int R, int LB>
+hbl_status launch_nfq_tc2(const NfqArgs& a, cudaStream_t s) {
+  static SmemLimit lim;
+  auto* k = norm_fht_quant_tc2_kernel<QM, R, LB>;
+  cudaError_t e = allow_smem(k, kN2Smem, lim);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaLaunchConfig_t cfg = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int sms = device_sms(dev);
+  const int groups = (a.M + R - 1) / R;
+  cfg.gridDim = dim3(groups < sms ? groups : sms, 1, 1);  // one CTA per SM
+  cfg.blockDim = dim3(kN2Threads, 1, 1);
+  cfg.dynamicSmemBytes = kN2Smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may overlap the kernel before
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, k, a);
+  if (e != cudaSuccess) return cuda_fail(e);
+  HBL_CHECK_LAUNCH();
+  return HBL_OK;
+}
+
 // No transform (blocks of one feature): up to E features per thread, tpr threads per row (a
 // multiple of 32, at most 1024, tpr * E >= K), and at least 256 threads per CTA.
 template <int E>
@@ -289,9 +316,18 @@ hbl_status run_nfq(const void* X, const float* gain, int M, int K, int had_block
   if (gain == nullptr) {
     auto tc = [&](auto rc, auto lc) -> hbl_status {
       constexpr int RR = decltype(rc)::value, LL = decltype(lc)::value;
-      if (quant == 0) return launch_nfq_tc<0, RR, LL>(a, stream);
-      if (quant == 1) return launch_nfq_tc<1, RR, LL>(a, stream);
-      return launch_nfq_tc<2, RR, LL>(a, stream);
+      // groups of 2 or 4 rows: two sets of eight consumer warps per SM (each row half of a group
+      // to four warps); one row of 16384 or a block-diagonal row: the 4-warp kernel (split in
+      // halves, the 16384-point rows need a TMEM exchange for k bit 13 and ran slower)
+      if constexpr (RR > 1) {
+        if (quant == 0) return launch_nfq_tc2<0, RR, LL>(a, stream);
+        if (quant == 1) return launch_nfq_tc2<1, RR, LL>(a, stream);
+        return launch_nfq_tc2<2, RR, LL>(a, stream);
+      } else {
+        if (quant == 0) return launch_nfq_tc<0, RR, LL>(a, stream);
+        if (quant == 1) return launch_nfq_tc<1, RR, LL>(a, stream);
+        return launch_nfq_tc<2, RR, LL>(a, stream);
+      }
     };
     using std::integral_constant;
     if (nb == 1 && L == 12) return tc(integral_constant<int, 4>{}, integral_constant<int, 12>{});
