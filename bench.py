@@ -56,7 +56,9 @@ def nfq_kernel(K, had_block):
     """Name of the fused activation kernel hbl_norm_fht_quant runs (no gain)."""
     if had_block == 1:
         return "norm_quant"
-    if had_block == 0 and K in (4096, 8192, 16384):
+    if had_block == 0 and K in (4096, 8192):
+        return "norm_fht_quant_tc2"
+    if had_block == 0 and K == 16384:
         return "norm_fht_quant_tc"
     if had_block == 256 and K <= 16384 and K & (K - 1):
         return "norm_fht_quant_tc"
