@@ -52,16 +52,17 @@ def product_kernel(M):
     return ("gemm_swap", "gemm_swap.cuh") if M <= 256 else ("gemm_tc2", "gemm_tc2.cuh")
 
 
-def nfq_kernel(K, had_block):
-    """Name of the fused activation kernel hbl_norm_fht_quant runs (no gain)."""
+def nfq_kernel(K, had_block, M):
+    """Name of the fused activation kernel hbl_norm_fht_quant runs on M rows (no gain): the
+    tensor-core kernels from 17 rows of 16384 features, 65 rows of 8192 and 257 rows otherwise."""
     if had_block == 1:
         return "norm_quant"
-    if had_block == 0 and K in (4096, 8192):
-        return "norm_fht_quant_tc2"
     if had_block == 0 and K == 16384:
-        return "norm_fht_quant_tc"
+        return "norm_fht_quant_tc" if M >= 17 else "norm_fht_quant"
+    if had_block == 0 and K in (4096, 8192):
+        return "norm_fht_quant_tc2" if M >= (65 if K == 8192 else 257) else "norm_fht_quant"
     if had_block == 256 and K <= 16384 and K & (K - 1):
-        return "norm_fht_quant_tc"
+        return "norm_fht_quant_tc" if M >= 257 else "norm_fht_quant"
     return "norm_fht_quant"
 
 
@@ -463,7 +464,7 @@ def run_ours(args, world, rank, local):
         sp = L["spec"]
         nfq_bytes = act_bytes(sp.M, sp.K, 4)
         gemm_ops = 2.0 * sp.M * sp.N * sp.K
-        kern.append({"kernel": f"{nfq_kernel(sp.K, sp.had_block)}[{sp.name}]", "ms": per[2 * i], "bound": "hbm",
+        kern.append({"kernel": f"{nfq_kernel(sp.K, sp.had_block, sp.M)}[{sp.name}]", "ms": per[2 * i], "bound": "hbm",
                      "achieved": nfq_bytes / (per[2 * i] / 1e3) / 1e9, "unit": "GB/s",
                      "frac": nfq_bytes / (per[2 * i] / 1e3) / 1e9 / hbm, "algorithmic_bytes": nfq_bytes,
                      "moved_bytes": act_container_bytes(sp.M, sp.K),
@@ -639,7 +640,7 @@ def time_configs(dev, hbm, int8_peak, reps=20):
         ops = 2.0 * M * N * K
         out.append({
             "config": label, "M": M, "K": K, "N": N, "had_block": spec.had_block,
-            "activation": {"kernel": nfq_kernel(K, spec.had_block), "us": res["act"], "bound": "hbm",
+            "activation": {"kernel": nfq_kernel(K, spec.had_block, M), "us": res["act"], "bound": "hbm",
                            "algorithmic_bytes": ab, "moved_bytes": act_container_bytes(M, K),
                            "GBps": ab / res["act"] / 1e3, "frac": ab / res["act"] / 1e3 / hbm},
             "product": {"kernel": product_kernel(M)[0], "us": res["prod"], "bound": "tensor",
@@ -690,12 +691,13 @@ def run_profile_activation(name, M):
     st = hbl.hbl_device_status()
     if st != hbl.HBL_OK:
         raise RuntimeError(hbl.hbl_status_string(st))
-    print(f"activation {nfq_kernel(spec.K, spec.had_block)}: {name} M={M} K={spec.K}, 3 launches", flush=True)
+    print(f"activation {nfq_kernel(spec.K, spec.had_block, M)}: {name} M={M} K={spec.K}, 3 launches", flush=True)
 
 
-def run_profile_forward(M, name="wdown_7b_a4"):
-    """Runs hbl_forward three times on one workload with M tokens (one token of K <= 8192 is the
-    fused decode kernel: one launch per layer); an ncu target, no bench line."""
+def run_profile_forward(M, name="wdown_7b_a4", decode=False):
+    """Runs hbl_forward three times on one workload with M tokens (with `decode`, one token through
+    hbl_forward_decode: the fused decode kernel, one launch per layer); an ncu target, no bench
+    line."""
     import torch
 
     import hadamard_bit_quant_hbl_b200 as hbl
@@ -705,7 +707,10 @@ def run_profile_forward(M, name="wdown_7b_a4"):
     X = torch.from_numpy(inputs.activations(spec).view(np.int16)).cuda().view(torch.bfloat16)
     packed, alpha = hbl.hbl_pack_weights(torch.from_numpy(inputs.weights(spec)).cuda())
     for _ in range(3):
-        hbl.hbl_forward(X, packed, alpha, spec.N, None, 0, hbl.HBL_Q_A4_ABSMEAN, out_dtype=hbl.HBL_OUT_BF16)
+        if decode:
+            hbl.hbl_forward_decode(X, packed, alpha, spec.N, None, 0, hbl.HBL_Q_A4_ABSMEAN, out_dtype=hbl.HBL_OUT_BF16)
+        else:
+            hbl.hbl_forward(X, packed, alpha, spec.N, None, 0, hbl.HBL_Q_A4_ABSMEAN, out_dtype=hbl.HBL_OUT_BF16)
     torch.cuda.synchronize()
     st = hbl.hbl_device_status()
     if st != hbl.HBL_OK:
@@ -777,7 +782,7 @@ def run_activation_only(reps=50):
         if st != hbl.HBL_OK:
             raise RuntimeError(hbl.hbl_status_string(st))
         us = e0.elapsed_time(e1) / reps * 1000
-        kern = nfq_kernel(K, spec.had_block)
+        kern = nfq_kernel(K, spec.had_block, M)
         ab = act_bytes(M, K, spec.abits)
         print(f"{kern:18s} {name:18s} M={M:5d} K={K:6d} had_block={spec.had_block:4d} {us:8.1f} us "
               f"{ab / us / 1e3:7.1f} GB/s {ab / us / 1e3 / peak:6.3f} of {peak_src} HBM on a4 algorithmic bytes "
@@ -837,6 +842,9 @@ def main():
     ap.add_argument("--profile-forward", nargs="+", metavar=("M", "WORKLOAD"),
                     help="only run hbl_forward three times with M tokens on a workload (default the 7B Wdown; "
                          "an ncu target)")
+    ap.add_argument("--profile-decode", default=None, metavar="WORKLOAD",
+                    help="only run hbl_forward_decode (one token, one launch) three times on a workload "
+                         "(an ncu target)")
     ap.add_argument("--profile-qkv", type=int, default=0, metavar="M",
                     help="only run the QKV quantiser three times on M tokens x 32 heads x 128 (an ncu target)")
     args = ap.parse_args()
@@ -851,6 +859,9 @@ def main():
         return
     if args.profile_forward:
         run_profile_forward(int(args.profile_forward[0]), *args.profile_forward[1:2])
+        return
+    if args.profile_decode:
+        run_profile_forward(1, args.profile_decode, decode=True)
         return
     if args.profile_product:
         run_profile_product(args.profile_product)

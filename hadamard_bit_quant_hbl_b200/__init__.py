@@ -23,7 +23,7 @@ __all__ = [
     "hbl_status_string", "hbl_device_status", "hbl_selftest_timeout", "hbl_packed_weights_bytes", "hbl_pack_weights_workspace",
     "hbl_pack_weights", "hbl_pack_weights_rotated", "hbl_pack_weights_rotated_workspace", "hbl_pack_ternary",
     "hbl_norm_fht_quant", "hbl_ternary_gemm",
-    "hbl_forward_workspace", "hbl_forward", "codes_row_bytes",
+    "hbl_forward_workspace", "hbl_forward", "hbl_forward_decode", "codes_row_bytes",
     "hbl_qkv_codes_bytes", "hbl_qkv_quant", "hbl_qkv_dequant",
 ]
 
@@ -68,6 +68,8 @@ _SIGNATURES = {
     "hbl_forward": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_size_t, _c_float, _c_int, _c_int, _c_int,
                              _c_int, _c_int, _c_float, _c_float, _c_void_p, _c_size_t, _c_void_p, _c_int,
                              _c_void_p]),
+    "hbl_forward_decode": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_size_t, _c_float, _c_int, _c_int, _c_int,
+                                    _c_int, _c_float, _c_float, _c_void_p, _c_int, _c_void_p]),
 }
 
 
@@ -255,6 +257,23 @@ def hbl_forward(X, packed, alpha: float, N: int, gain=None, had_block: int = 0, 
     _check(lib().hbl_forward(_ptr(X), _ptr(gain), _ptr(packed), packed.numel(), float(alpha), M, K, N, had_block,
                              quant, float(eps_norm), float(eps_q), _ptr(workspace), workspace.numel(), _ptr(Y),
                              out_dtype, _stream(stream, X)), "hbl_forward")
+    return Y
+
+
+def hbl_forward_decode(X, packed, alpha: float, N: int, gain=None, had_block: int = 0, quant: int = HBL_Q_A4_ABSMEAN,
+                       eps_norm: float = 1e-6, eps_q: float = 0.0, Y=None, out_dtype: int = HBL_OUT_F32, stream=None):
+    """One token of the forward in one launch, no workspace: bf16 X [1, K] (K a power of two up to
+    8192) with packed weights. Returns Y [1, N]."""
+    import torch
+
+    M, K = X.shape
+    if M != 1:
+        raise ValueError("hbl_forward_decode takes one token")
+    if Y is None:
+        Y = torch.empty((1, N), dtype=torch.float32 if out_dtype == HBL_OUT_F32 else torch.bfloat16, device=X.device)
+    _check(lib().hbl_forward_decode(_ptr(X), _ptr(gain), _ptr(packed), packed.numel(), float(alpha), K, N, had_block,
+                                    quant, float(eps_norm), float(eps_q), _ptr(Y), out_dtype, _stream(stream, X)),
+           "hbl_forward_decode")
     return Y
 
 

@@ -313,7 +313,17 @@ hbl_status run_nfq(const void* X, const float* gain, int M, int K, int had_block
   // one row per group. (It also serves one block of 2^11 correctly; an earlier version of its
   // per-row epilogue measured slower there than the CUDA-core kernel, 12.5 against 7.1 us on
   // 2048 x 2048, so 2^11 stays on CUDA cores until measured again.)
-  if (gain == nullptr) {
+  // Few rows stay on the CUDA-core kernel: a tensor-core launch holds whole SMs (one or two CTAs
+  // of 66-164 KB of shared memory and all of TMEM) and its setup (H in shared memory, the TMEM
+  // allocation) is not amortised, while the small kernel leaves room for the product that follows
+  // to start streaming its weights early (programmatic launch). Thresholds from B200 timings of
+  // the forward in a CUDA graph: 16384 features up to 16 rows (Wdown 7B at 1 / 16 tokens: 10.9 /
+  // 15.0 against 11.5 / 15.6 us), 4096 up to 256 rows (Wo 7B at 1 / 16 / 64 tokens, two kernels:
+  // 6.1 / 7.2 / 10.0 against 8.7 / 9.2 / 11.6 us; alone at 256 rows 5.8 against 7.3 us), 8192 up
+  // to 64 (alone: equal at 64 rows, the tensor cores ahead at 256), block-diagonal rows up to 256
+  // (alone at 256 rows: 6.0 against 10.5 us).
+  const int tc_min_rows = (nb == 1 && L == 14) ? 17 : ((nb == 1 && L == 13) ? 65 : 257);
+  if (gain == nullptr && M >= tc_min_rows) {
     auto tc = [&](auto rc, auto lc) -> hbl_status {
       constexpr int RR = decltype(rc)::value, LL = decltype(lc)::value;
       // groups of 2 or 4 rows: two sets of eight consumer warps per SM (each row half of a group
@@ -620,8 +630,7 @@ hbl_status run_swap(const void* codes_i8, const void* w2, const TcArgs& t, cudaS
 // codes up to 8 (the tensor-core kernels read one int8 per code).
 constexpr int kDecodeMaxM = 4;
 constexpr int kDecodeMaxMPacked = 8;
-// hbl_forward fuses the activation side into the decode product up to these sizes.
-constexpr int kFusedMaxM = 1;
+// hbl_forward_decode fuses the activation side into the decode product up to this width.
 constexpr int kFusedMaxK = 8192;
 
 hbl_status run_gemm(const void* codes, int fmt, int abits, const float* s_x, const void* packed, float alpha,
@@ -969,43 +978,6 @@ hbl_status hbl_forward(const void* X, const float* gain, const void* packed, siz
   if (ws_bytes < hbl_forward_workspace(M, K, quant)) return HBL_EINVAL;
   if (packed_bytes < blob_layout(K, N).total || !aligned(packed, 256) || !aligned(Y, 16)) return HBL_EINVAL;
   const int abits = quant == HBL_Q_A8_ABSMAX ? 8 : 4;
-  // One token (decode) of a power-of-two K up to kFusedMaxK: one launch computes the activation
-  // side of each CTA's slice of K in the product kernel itself (one transform block, blocks of a
-  // power of two, or none); the codes never leave the SM. With more tokens or wider rows every CTA
-  // repeats more of the row's transform than the separate activation kernel costs (measured on
-  // B200, Wo 4096 -> 4096: 8.0 against 9.2 us at one token, 16.1 against 10.8 us at four; Wdown
-  // 16384 -> 4096 at one token: 12.3 against 11.8 us), so those take the two-kernel path.
-  if (M <= kFusedMaxM && K <= kFusedMaxK && is_pow2(K)) {
-    const int n = had_block == 0 ? K : had_block;
-    const bool hb_ok = n == 1 || (is_pow2(n) && n >= 256 && n <= 16384 && (K % n) == 0);
-    if (hb_ok) {
-      if (quant != HBL_Q_A8_ABSMAX && quant != HBL_Q_A4_ABSMEAN && quant != HBL_Q_A4_ABSMAX) return HBL_EUNSUPPORTED;
-      if (!(eps_norm >= 0.f) || !(eps_q >= 0.f)) return HBL_EINVAL;
-      if (!aligned(X, 16) || (gain && !aligned(gain, 4))) return HBL_EINVAL;
-      if (out_dtype != HBL_OUT_F32 && out_dtype != HBL_OUT_BF16) return HBL_EINVAL;
-      const BlobLayout bl = blob_layout(K, N);
-      DecodeArgs d;
-      d.m0 = 0;
-      d.codes = nullptr;
-      d.packed4 = 0;
-      d.s_x = nullptr;
-      d.w2 = reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(packed) + bl.off0);
-      d.alpha = alpha;
-      d.M = M;
-      d.N = N;
-      d.K = K;
-      d.Y = Y;
-      d.out_bf16 = out_dtype == HBL_OUT_BF16;
-      d.acc_debug = nullptr;
-      d.X = static_cast<const uint16_t*>(X);
-      d.gain = gain;
-      d.hb = n;
-      d.quant = (int)quant;
-      d.eps_norm = eps_norm;
-      d.eps_q = eps_q;
-      return run_decode(d, true, reinterpret_cast<cudaStream_t>(stream));
-    }
-  }
   const hbl_codes_fmt fmt = HBL_CODES_I8;  // both tensor-core products read one int8 per code
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* codes = ws;
@@ -1014,6 +986,49 @@ hbl_status hbl_forward(const void* X, const float* gain, const void* packed, siz
   if (st != HBL_OK) return st;
   return hbl_ternary_gemm(codes, fmt, abits, s_x, packed, packed_bytes, alpha, M, N, K, Y, out_dtype, nullptr,
                           stream);
+}
+
+// One token in one launch (the decode product computes its own codes): see hbl.h. Measured on
+// B200 (Wo 4096 -> 4096, one token): 8.0 us against 9.2 us for two launches while the activation
+// of few rows ran on the tensor-core kernel, 7.5 against 6.1 us since it runs on CUDA cores; with
+// more tokens or wider rows every CTA repeats more of the row's transform than the separate
+// activation kernel costs (16.1 against 10.8 us at four tokens; Wdown 16384 -> 4096 at one token
+// 12.3 against 11.8 us), so the entry takes one token of K <= kFusedMaxK only.
+hbl_status hbl_forward_decode(const void* X, const float* gain, const void* packed, size_t packed_bytes,
+                              float alpha, int K, int N, int had_block, hbl_quant quant, float eps_norm,
+                              float eps_q, void* Y, hbl_out_dtype out_dtype, hbl_stream_t stream) {
+  if (!X || !packed || !Y) return HBL_EINVAL;
+  if (!dims_ok(1, K) || N < 8 || (N % 8)) return HBL_EINVAL;
+  if (packed_bytes < blob_layout(K, N).total || !aligned(packed, 256) || !aligned(Y, 16)) return HBL_EINVAL;
+  if (K > kFusedMaxK || !is_pow2(K)) return HBL_EUNSUPPORTED;
+  const int n = had_block == 0 ? K : had_block;
+  const bool hb_ok = n == 1 || (is_pow2(n) && n >= 256 && n <= 16384 && (K % n) == 0);
+  if (!hb_ok) return HBL_EUNSUPPORTED;
+  if (quant != HBL_Q_A8_ABSMAX && quant != HBL_Q_A4_ABSMEAN && quant != HBL_Q_A4_ABSMAX) return HBL_EUNSUPPORTED;
+  if (!(eps_norm >= 0.f) || !(eps_q >= 0.f)) return HBL_EINVAL;
+  if (!aligned(X, 16) || (gain && !aligned(gain, 4))) return HBL_EINVAL;
+  if (out_dtype != HBL_OUT_F32 && out_dtype != HBL_OUT_BF16) return HBL_EINVAL;
+  const BlobLayout bl = blob_layout(K, N);
+  DecodeArgs d;
+  d.m0 = 0;
+  d.codes = nullptr;
+  d.packed4 = 0;
+  d.s_x = nullptr;
+  d.w2 = reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(packed) + bl.off0);
+  d.alpha = alpha;
+  d.M = 1;
+  d.N = N;
+  d.K = K;
+  d.Y = Y;
+  d.out_bf16 = out_dtype == HBL_OUT_BF16;
+  d.acc_debug = nullptr;
+  d.X = static_cast<const uint16_t*>(X);
+  d.gain = gain;
+  d.hb = n;
+  d.quant = (int)quant;
+  d.eps_norm = eps_norm;
+  d.eps_q = eps_q;
+  return run_decode(d, true, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

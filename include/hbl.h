@@ -159,9 +159,12 @@ hbl_status hbl_pack_ternary(const int8_t* t, int K, int N, void* packed, size_t 
  *            is 0 gives q = 0, s = 0. Rounding: nearest, ties to even. The kernels transform and
  *            decide in fp32, so a value within fp32 rounding of a .5 boundary may land on
  *            either side of it (a one-step code difference from an exact evaluation).
- * Kernels: one block of 4096, 8192 or 16384 features without gain runs the H_128 Kronecker factor of
- * the transform on the tensor cores and the rest on CUDA cores; had_block = 1 runs a streaming
- * norm-and-quantise kernel; every other shape runs the CUDA-core transform. Both give the same codes up to the rounding-order ties the parity tests allow.
+ * Kernels: without gain, one block of 16384 features from 17 rows, of 8192 from 65 rows, of 4096
+ * from 257 rows, and blocks of 256 in rows that are not a power of two from 257 rows run the H_128
+ * (or I_4 (x) H_32) Kronecker factor of the transform on the tensor cores and the rest on CUDA
+ * cores; had_block = 1 runs a streaming norm-and-quantise kernel; every other shape, and fewer
+ * rows, runs the CUDA-core transform. All give the same codes up to the rounding-order ties the
+ * parity tests allow.
  *
  *   X       device bf16 [M][K], 16-byte aligned
  *   gain    device fp32 [K] or NULL
@@ -202,11 +205,6 @@ hbl_status hbl_ternary_gemm(const void* codes, hbl_codes_fmt fmt, int abits, con
 
 /* ---------------------------------------------------------------------------------------
  * The whole layer forward: hbl_norm_fht_quant into `workspace`, then hbl_ternary_gemm.
- * For one token (M = 1) with K a power of two up to 8192 (had_block 0, 1, or a power of two)
- * it is one launch instead: the decode product computes the codes of each CTA's slice of K from
- * the bf16 row itself (the transform's stages across slices as signed sums of the row's slices,
- * the row statistics reduced over the CTA cluster), and writes nothing to `workspace`. The
- * result is the same layer, up to the one-step code flips any two fp32 evaluations may differ by.
  *   workspace  device scratch, ws_bytes >= hbl_forward_workspace(M, K, quant), 256-byte aligned
  * Asynchronous. */
 size_t hbl_forward_workspace(int M, int K, hbl_quant quant);
@@ -215,6 +213,22 @@ hbl_status hbl_forward(const void* X, const float* gain, const void* packed, siz
                        float alpha, int M, int K, int N, int had_block, hbl_quant quant,
                        float eps_norm, float eps_q, void* workspace, size_t ws_bytes, void* Y,
                        hbl_out_dtype out_dtype, hbl_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * One token of the layer forward (M = 1) in one launch and with no workspace: the decode
+ * product computes the codes of each CTA's slice of K from the bf16 row itself (the transform's
+ * stages across slices as signed sums of the row's slices, read from L2; the row statistics
+ * reduced over the CTA cluster), so nothing between the row and Y reaches device memory. Same
+ * layer and arguments as hbl_forward with M = 1, up to the one-step code flips any two fp32
+ * evaluations may differ by. K a power of two up to 8192; had_block 0, 1, or a power of two from
+ * 256 dividing K; else HBL_EUNSUPPORTED. (hbl_forward runs one token as two launches, the
+ * few-row activation kernel and the decode product, which measured faster on B200: Wo 4096 ->
+ * 4096 6.1 against 7.5 us.)
+ *   X   device bf16 [K], 16-byte aligned;   Y   device [N] of out_dtype, 16-byte aligned
+ * Asynchronous. */
+hbl_status hbl_forward_decode(const void* X, const float* gain, const void* packed, size_t packed_bytes,
+                              float alpha, int K, int N, int had_block, hbl_quant quant, float eps_norm,
+                              float eps_q, void* Y, hbl_out_dtype out_dtype, hbl_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------
  * Low-bit attention states: QKV quantised after RoPE to unsigned integers per head.

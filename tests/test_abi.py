@@ -95,6 +95,31 @@ def test_gemm_and_forward_reject_bad_arguments(L):
     assert fw(FAKE, None, FAKE, nbytes, 1.0, 4, 1024, 64, 0, 1, 1e-6, 0.0, None, ws, FAKE, 0, None) == hbl.HBL_EINVAL
 
 
+def test_forward_decode_rejects_bad_arguments(L):
+    # every call below has at least one invalid argument, so none reaches a kernel
+    fd = L.hbl_forward_decode
+    nb = lambda K, N: hbl.hbl_packed_weights_bytes(K, N)  # noqa: E731
+    ok = dict(X=FAKE, gain=None, packed=FAKE, pb=nb(1024, 64), alpha=1.0, K=1024, N=64, hb=0, quant=1,
+              en=1e-6, eq=0.0, Y=FAKE, od=0)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return fd(a["X"], a["gain"], a["packed"], a["pb"], a["alpha"], a["K"], a["N"], a["hb"], a["quant"],
+                  a["en"], a["eq"], a["Y"], a["od"], None)
+
+    assert call(X=None) == hbl.HBL_EINVAL
+    assert call(Y=None, quant=9) == hbl.HBL_EINVAL
+    assert call(N=60, quant=9) == hbl.HBL_EINVAL                       # N % 8
+    assert call(pb=nb(1024, 64) - 1, quant=9) == hbl.HBL_EINVAL       # blob too small
+    assert call(K=16384, pb=nb(16384, 64)) == hbl.HBL_EUNSUPPORTED     # wider than one launch takes
+    assert call(K=3072, pb=nb(3072, 64)) == hbl.HBL_EUNSUPPORTED       # not a power of two
+    assert call(hb=128) == hbl.HBL_EUNSUPPORTED                         # transform block below 256
+    assert call(quant=9) == hbl.HBL_EUNSUPPORTED
+    assert call(en=-1.0) == hbl.HBL_EINVAL
+    assert call(X=FAKE + 2) == hbl.HBL_EINVAL                           # misaligned
+    assert call(od=7) == hbl.HBL_EINVAL
+
+
 def test_pack_rejects_bad_arguments(L):
     alpha = ctypes.c_float(0)
     nbytes = hbl.hbl_packed_weights_bytes(512, 64)
