@@ -51,7 +51,6 @@
 
 #include "common.cuh"
 #include "gemm_tc.cuh"
-#include "gemm_tc2.cuh"
 
 namespace hbl {
 
