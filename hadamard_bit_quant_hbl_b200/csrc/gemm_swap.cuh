@@ -13,9 +13,9 @@
 // into int8 in registers and store it with tcgen05.st, so the widened weights (4x the 2-bit bytes)
 // never pass through shared memory, whose bandwidth bounded an earlier form of this kernel. A
 // widened byte is 64 t rather than t (two instructions per 4 codes: the code plane shifted to bits
-// 6..7 and offset so that c' = t + 1 in {0, 1, 2} becomes the sign-magnitude pattern of 64 t), so
-// the MMAs accumulate 64 sum t q, divided back exactly in the epilogue (|64 sum t q| < 2^29 for
-// K <= 32768).
+// 6..7 plus 0xc0 per byte, masked to bits 6..7, turns c' = t + 1 in {0, 1, 2} into the int8 bytes
+// 0xc0, 0x00, 0x40; the carries only reach the masked-off bits), so the MMAs accumulate
+// 64 sum t q, divided back exactly in the epilogue (|64 sum t q| <= 2^28 for K <= 32768).
 //
 // A cluster of S CTAs shares one 128-feature tile and splits K: CTA r owns a contiguous run of
 // 128-wide k-blocks, processed in batches of BK k-blocks. Its partial sums end in its own shared
@@ -316,8 +316,8 @@ gemm_swap_kernel(const __grid_constant__ CUtensorMap mapA, const SwapArgs a) {
     } else if (warp >= 4) {
       // ---------------- widen: thread = weight row (lane quarter q = warp % 4); the 128 codes of
       // a k-block (8 words, 16 codes each: k = 16c + 4s + b at bits 8b + 2s, c' = t + 1) become
-      // 32 columns of 4 int8, column 4c + s holding k = 16c + 4s + 0..3. Warp group g takes
-      // batches g, g + kSwW, ...
+      // 32 columns of 4 int8 bytes 64 t, column 4c + s holding k = 16c + 4s + 0..3. Warp group g
+      // takes batches g, g + kSwW, ...
       const int q = warp & 3, g = (warp - 4) >> 2;
       const int row = q * 32 + lane;
       const uint32_t t_lane = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)a.acc_cols;
