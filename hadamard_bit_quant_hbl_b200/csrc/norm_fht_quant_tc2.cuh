@@ -44,6 +44,8 @@ constexpr int kN2MaxRegs = 96;
 static_assert(5 * 32 * kN2MaxRegs <= 16384, "registers of the warps on one scheduler");
 static_assert(kN2Smem <= 227 * 1024, "shared memory");
 
+// Named barrier of one consumer set (its 256 threads; id 1 + set); the second form also returns,
+// in every thread, the OR of `pred` over the set (a uniform decision).
 __device__ __forceinline__ void set_bar(uint32_t id) {
   asm volatile("bar.sync %0, 256;" ::"r"(id) : "memory");
 }
