@@ -153,7 +153,10 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend="nccl"):
+    """Rank, world size and local rank from the launcher's environment; with more than one rank a
+    process group (NCCL on the GPUs; gloo for the host-side tests) with a short timeout, so that
+    ranks waiting for a lost peer end with an error instead of hanging."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -163,10 +166,31 @@ def dist_setup(n_gpus):
         import torch
         import torch.distributed as dist
 
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return world, rank, local
+
+
+def max_over_ranks(value, world, device=None):
+    """The largest `value` over all ranks (a job takes as long as its slowest replica); the value
+    itself with one rank. Every rank must call it, in the same order."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank, world, ms_per_step):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's step time."""
+    return tokens_per_rank * world / (ms_per_step / 1e3)
 
 
 # ---------------------------------------------------------------- CPU oracle (reference arm)
@@ -385,13 +409,10 @@ def run_ours(args, world, rank, local):
             per[j] += marks[j].elapsed_time(marks[j + 1])
     per /= args.steps
     # per-kernel split of the first pair includes the launch of the nfq kernel of layer 0 only
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     ms_step = total_ms / args.steps
     tokens = M_TOKENS * world
-    value = tokens / (ms_step / 1e3)
+    value = job_throughput(M_TOKENS, world, ms_step)
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed
     # region. Steps are pipelined as a serving loop would: the host->device copy of step k+1 and
@@ -440,10 +461,7 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1) / e2e_steps
         del Xd, Yd
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
     h2d = sum(L["X"].numel() * 2 for L in layers)
     d2h = sum(L["Y"].numel() * 2 for L in layers)
 
