@@ -31,7 +31,7 @@
 //               commit to each of the slot's and the activation stage's "empty" barriers
 //   warp 2      TMA copies of the batch's activation tiles (Mt rows x 128 bytes per k-block,
 //               128-byte swizzle) into an NA-stage ring
-//   warp 3      s_x * alpha into shared memory for the epilogue; with nis = 2 (up to 64 tokens)
+//   warp 3      s_x * alpha into shared memory for the epilogue; with nis = 2 (up to 128 tokens)
 //               one thread also issues batches 1, 3, ... into the second accumulator: a small-N
 //               MMA occupies the tensor core for about 45 cycles, less than one thread needs to
 //               issue it while the widening warps share its scheduler
