@@ -18,7 +18,7 @@ import torch
 import oracle
 import hadamard_bit_quant_hbl_b200 as hbl
 from hadamard_bit_quant_hbl_b200 import inputs
-from formats import blob_offsets, code_flips, decode_blob, pack_int4, row_rel_err, unpack_int4
+from formats import code_flips, decode_blob, pack_int4, row_rel_err, unpack_int4
 
 pytestmark = pytest.mark.gpu
 
