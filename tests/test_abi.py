@@ -173,3 +173,11 @@ def test_qkv_quant_rejects_bad_arguments(L):
     d = hbl.lib().hbl_qkv_dequant
     assert d(None, FAKE, 1, 4, 128, 3, FAKE, None) == hbl.HBL_EINVAL
     assert d(FAKE, FAKE, 1, 4, 100, 3, FAKE, None) == hbl.HBL_EUNSUPPORTED
+
+
+def test_binding_forward_decode_takes_one_token():
+    import torch
+
+    X = torch.zeros((2, 1024), dtype=torch.bfloat16)  # host tensor: rejected before any library call
+    with pytest.raises(ValueError):
+        hbl.hbl_forward_decode(X, torch.zeros(16, dtype=torch.uint8), 1.0, 64)
